@@ -1,0 +1,44 @@
+// Internal launch functions behind the C ABI (host side, not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace qsa {
+
+cudaError_t launch_pool(const uint16_t *k_idx, int B, int64_t T, int Di, int64_t j0,
+                        int64_t j1, uint16_t *kp, cudaStream_t s, int num_sms);
+
+size_t index_topk_ws_bytes(int grid);
+int index_topk_grid(int num_sms);
+int index_topk_max_keep();
+cudaError_t launch_index_topk(const uint16_t *q_idx, const float *w, const uint16_t *kp,
+                              const int64_t *q_pos0, int B, int64_t Tq, int64_t n_blocks,
+                              int Hi, int Di, int kb, int32_t *sel, float *sel_score,
+                              void *ws, int grid, cudaStream_t s);
+
+size_t index_decode_ws_bytes(int B, int64_t n_blocks, int kb, int num_sms);
+int index_decode_merge_cap(int64_t n_blocks, int kb);  // -1: too many splits
+cudaError_t launch_index_topk_decode(const uint16_t *q_idx, const float *w, const uint16_t *kp,
+                                     const int32_t *seqlens, int B, int64_t n_blocks, int Hi,
+                                     int Di, int kb, int32_t *sel, float *sel_score, void *ws,
+                                     int num_sms, cudaStream_t s);
+
+int sparse_attn_blocks_per_stage(int Hkv);
+cudaError_t launch_sparse_attn_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                       const int32_t *sel, const int64_t *q_pos0, int B,
+                                       int64_t Tq, int64_t Tk, int Hq, int Hkv, int D, int kb,
+                                       float scale, uint16_t *o, float *lse, int num_sms,
+                                       cudaStream_t s);
+cudaError_t launch_split_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                const int32_t *seqlens, int64_t L_max, const int32_t *sel,
+                                int n_entries, int nsplit, int B, int Hq, int Hkv, int D,
+                                float scale, uint16_t *o, float *lse, float *part,
+                                void *status, int num_sms, cudaStream_t s);
+
+cudaError_t launch_dense_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
+                                 int64_t T, int Hq, int Hkv, int D, float scale, uint16_t *o,
+                                 float *lse, cudaStream_t s);
+
+}  // namespace qsa

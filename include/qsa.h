@@ -1,0 +1,221 @@
+/*
+ * qsa.h -- C ABI of libqsa, a B200 (sm_100a) implementation of the Qwen
+ * Sparse Attention (QSA) layer: micro-block pooling, a lightweight MQA
+ * indexer with top-k block selection, and exact softmax attention over the
+ * tokens of the selected blocks, for prefill and decode; plus dense causal
+ * GQA attention on the same tensors (the speed-up baseline).
+ *
+ * Sources (web pages about the Qwen3.8-Flash-Next architecture):
+ *   [ART]  "用125亿分之6的参数，打平3970亿的旗舰模型", section
+ *          "稀疏注意力：给检索建索引，也得先学会省纸".
+ *   [SUM]  "On the Design of Qwen3.8-Next Architecture: Evaluation,
+ *          Efficiency, and Training Stability", token-mixing paragraph.
+ *   [NEWS] "Qwen3.8-Flash发布并开源：6B激活参数背后，是Qwen4架构的第一次公开
+ *          亮相", section "二、架构 / 1. 注意力机制".
+ *
+ * Conventions, for every entry point:
+ *   - Tensor arguments are DEVICE pointers to contiguous row-major arrays
+ *     (last dimension innermost), 16-byte aligned, allocated and owned by the
+ *     caller.  bf16 tensors are passed as raw 16-bit patterns (qsa_bf16_t).
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  All work is enqueued asynchronously on it; the library never
+ *     allocates, frees or synchronises, except qsa_check_device_status.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and returned synchronously (QSA_ERR_INVALID_ARG / _UNSUPPORTED_SHAPE /
+ *     _WORKSPACE).  A device that is not sm_100 gives QSA_ERR_ARCH.  A failed
+ *     launch gives QSA_ERR_CUDA.
+ *   - Errors detected by a kernel (an out-of-range value read from a device
+ *     array) are recorded in the status word at the start of the workspace
+ *     and read back with qsa_check_device_status.  Kernels never trap.
+ *   - Workspace sizes from the *_workspace_size functions are byte counts;
+ *     0 is never returned for a valid shape (the status header is included).
+ *     SIZE_MAX means the arguments are invalid.
+ *   - Calls that share a workspace must be ordered on one stream.
+ *   - Supported shapes on the GPU: r = 4; D in {64, 128}; Di in {32, 64};
+ *     Hi in {1, 2, 4}; Hkv in {1, 2, 4}; G = Hq / Hkv in {1, 2, 4, 8};
+ *     budget a multiple of r with budget / r <= 1024.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QSA_API __attribute__((visibility("default")))
+#else
+#define QSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QSA_OK = 0,
+    QSA_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad ratio */
+    QSA_ERR_UNSUPPORTED_SHAPE = 2, /* valid but outside the GPU kernels' set */
+    QSA_ERR_WORKSPACE = 3,         /* workspace missing or too small */
+    QSA_ERR_ARCH = 4,              /* current device is not sm_100 */
+    QSA_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    QSA_ERR_TIMEOUT = 6,           /* a bounded device-side wait ran out */
+    QSA_ERR_DEVICE = 7             /* a kernel met an out-of-range input value */
+} qsa_status_t;
+
+typedef uint16_t qsa_bf16_t; /* raw bf16 bit pattern */
+
+/*
+ * Micro-block mean pooling [ART: consecutive tokens packed into a micro-block
+ * and mean-pooled into one representative key; SUM: compression ratio 4].
+ *
+ *   k_pooled[b, j, :] = bf16_rne( ((k[4j] + k[4j+1]) + (k[4j+2] + k[4j+3])) * 0.25 )
+ *
+ * with the sums in fp32, for every batch row b and every block j in
+ * [blk_begin, blk_end).  Other blocks of k_pooled are left untouched, so a
+ * decode loop pools exactly the block a new token completes.
+ *   k_idx    [B, T, Di] bf16   indexer keys (one shared key head)
+ *   k_pooled [B, T / r, Di] bf16
+ * Requires r == 4, Di % 8 == 0, 0 <= blk_begin <= blk_end <= T / r.
+ */
+QSA_API qsa_status_t qsa_pool(const qsa_bf16_t *k_idx, int B, int64_t T, int Di, int r,
+                      int64_t blk_begin, int64_t blk_end, qsa_bf16_t *k_pooled,
+                      void *stream);
+
+/*
+ * Indexer scores and top-k block selection for a run of query tokens
+ * [ART: a lightweight MQA indexer gives every micro-block a score and the
+ * highest-scoring blocks are kept; SUM: indexing cost O(n^2 / r), token
+ * budget 2048].
+ *
+ * Query t of batch row b sits at absolute position p = q_pos0[b] + t
+ * (q_pos0 == NULL: p = t).  Its candidates are the complete blocks
+ * j < c = floor(p / r), scored in fp32 as
+ *     s(t, j) = sum_h w[b, t, h] * max(0, q_idx[b, t, h, :] . k_pooled[b, j, :]).
+ * It keeps the kb - 1 best candidates (score descending, lower block index
+ * first on equal scores), adds its own block c, and writes them ascending,
+ * padded with -1, kb = budget / r entries per query.
+ *   q_idx     [B, Tq, Hi, Di] bf16
+ *   w         [B, Tq, Hi] fp32 per-token head weights
+ *   k_pooled  [B, n_blocks, Di] bf16
+ *   q_pos0    [B] int64 device array, or NULL
+ *   sel       [B, Tq, kb] int32 (output)
+ *   sel_score [B, Tq, kb] fp32 (output, may be NULL): the score of each kept
+ *             block; +inf for the own block, -inf for padding
+ *   ws        device workspace of at least qsa_index_topk_workspace_size(...)
+ *             bytes; its first 256 bytes hold the device status word
+ * A position whose floor(p / r) exceeds n_blocks is clamped to n_blocks and
+ * recorded as QSA_ERR_DEVICE in the status word.
+ */
+QSA_API size_t qsa_index_topk_workspace_size(int B, int64_t Tq, int64_t n_blocks, int Hi,
+                                     int Di, int r, int budget);
+QSA_API qsa_status_t qsa_index_topk(const qsa_bf16_t *q_idx, const float *w,
+                            const qsa_bf16_t *k_pooled, const int64_t *q_pos0,
+                            int B, int64_t Tq, int64_t n_blocks, int Hi, int Di,
+                            int r, int budget, int32_t *sel, float *sel_score,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Decode-step selection: one new query per sequence at p = seqlens[b] - 1,
+ * same scores, ranking and output as qsa_index_topk with Tq = 1, but the
+ * candidates of each sequence are split across many CTAs and merged, so a
+ * batch of 64 sequences fills the GPU.
+ *   q_idx [B, Hi, Di] bf16, w [B, Hi] fp32, k_pooled [B, n_blocks, Di] bf16,
+ *   seqlens [B] int32 device array (1 <= seqlens[b] and
+ *   floor((seqlens[b] - 1) / r) <= n_blocks, else clamped and recorded as
+ *   QSA_ERR_DEVICE), sel [B, kb] int32, sel_score [B, kb] fp32 (nullable).
+ */
+QSA_API size_t qsa_index_topk_decode_workspace_size(int B, int64_t n_blocks, int r,
+                                            int budget);
+QSA_API qsa_status_t qsa_index_topk_decode(const qsa_bf16_t *q_idx, const float *w,
+                                   const qsa_bf16_t *k_pooled,
+                                   const int32_t *seqlens, int B,
+                                   int64_t n_blocks, int Hi, int Di, int r,
+                                   int budget, int32_t *sel, float *sel_score,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Sparse prefill attention [ART: the selected blocks are expanded back into
+ * their original tokens, which take part in the real attention; NEWS:
+ * full-precision attention over the selected blocks only].
+ *
+ * Query t of batch row b at position p = q_pos0[b] + t (q_pos0 NULL: p = t)
+ * attends to the tokens S = { r*j + i : j in sel[b, t, :], j >= 0,
+ * 0 <= i < r, r*j + i <= p }.  For head h, with g = h / (Hq / Hkv):
+ *     o[b, t, h] = sum_{u in S} softmax_u(scale * q[b, t, h] . k[b, u, g]) v[b, u, g]
+ *     lse[b, t, h] = ln sum_{u in S} exp(scale * q[b, t, h] . k[b, u, g])
+ * Logits, softmax statistics and accumulation in fp32; the probabilities are
+ * rounded to bf16 for the P.V product; o rounded to bf16.
+ *   q [B, Tq, Hq, D] bf16; k, v [B, Tk, Hkv, D] bf16 (p < Tk required);
+ *   sel [B, Tq, kb] int32 (any order; entries < 0 or with r*j > p ignored);
+ *   q_pos0 [B] int64 or NULL; o [B, Tq, Hq, D] bf16; lse [B, Tq, Hq] fp32
+ *   or NULL.  An empty token set gives o = 0 and lse = -inf.
+ */
+QSA_API qsa_status_t qsa_sparse_attn_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                     const qsa_bf16_t *v, const int32_t *sel,
+                                     const int64_t *q_pos0, int B, int64_t Tq,
+                                     int64_t Tk, int Hq, int Hkv, int D, int r,
+                                     int budget, float scale, qsa_bf16_t *o,
+                                     float *lse, void *stream);
+
+/*
+ * Sparse decode attention: the same definition for one query per sequence at
+ * p = seqlens[b] - 1, over the KV caches.  The selected tokens are split
+ * across CTAs and the partial results merged with their log-sum-exp.
+ *   q [B, Hq, D] bf16; k_cache, v_cache [B, L_max, Hkv, D] bf16;
+ *   seqlens [B] int32 (1..L_max, else the row is treated as empty and
+ *   QSA_ERR_DEVICE recorded); sel [B, kb] int32; o [B, Hq, D] bf16;
+ *   lse [B, Hq] fp32 or NULL.
+ */
+QSA_API size_t qsa_sparse_attn_decode_workspace_size(int B, int Hq, int D, int r,
+                                             int budget);
+QSA_API qsa_status_t qsa_sparse_attn_decode(const qsa_bf16_t *q, const qsa_bf16_t *k_cache,
+                                    const qsa_bf16_t *v_cache,
+                                    const int32_t *seqlens, int64_t L_max,
+                                    const int32_t *sel, int B, int Hq, int Hkv,
+                                    int D, int r, int budget, float scale,
+                                    qsa_bf16_t *o, float *lse, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/*
+ * Dense causal GQA attention, prefill: every query t attends to all tokens
+ * u <= t (the full-attention layer QSA replaces; speed-up baseline).
+ *   q [B, T, Hq, D], k, v [B, T, Hkv, D], o [B, T, Hq, D] bf16;
+ *   lse [B, T, Hq] fp32 or NULL.
+ */
+QSA_API qsa_status_t qsa_dense_gqa_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                   const qsa_bf16_t *v, int B, int64_t T, int Hq,
+                                   int Hkv, int D, float scale, qsa_bf16_t *o,
+                                   float *lse, void *stream);
+
+/*
+ * Dense GQA attention, decode: one query per sequence over all seqlens[b]
+ * cached tokens, split across CTAs and merged by log-sum-exp.
+ */
+QSA_API size_t qsa_dense_gqa_decode_workspace_size(int B, int64_t L_max, int Hq, int D);
+QSA_API qsa_status_t qsa_dense_gqa_decode(const qsa_bf16_t *q, const qsa_bf16_t *k_cache,
+                                  const qsa_bf16_t *v_cache,
+                                  const int32_t *seqlens, int64_t L_max, int B,
+                                  int Hq, int Hkv, int D, float scale,
+                                  qsa_bf16_t *o, float *lse, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, reads the status word kernels recorded at the start
+ * of `ws`, clears it, and returns it (QSA_OK if nothing was recorded).  The
+ * word is sticky: it keeps the first error recorded by any call that used
+ * this workspace since the last check.  A new workspace must have its first
+ * 256 bytes zeroed once before first use (this function leaves them zero).
+ */
+QSA_API qsa_status_t qsa_check_device_status(void *ws, void *stream);
+
+/* Static description of a status code. */
+QSA_API const char *qsa_status_string(qsa_status_t status);
+
+/* Library version, "major.minor.patch". */
+QSA_API const char *qsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */
