@@ -31,6 +31,7 @@
  *     blocks kb = budget / r includes the own block.
  *   - the selection is output ascending, padded with -1.
  *   - attention scale = caller-supplied (1/sqrt(D) in every workload).
+ *   - an empty token set gives o = 0 and lse = -inf.
  *
  * "Parity unpinned": the scoring form itself.  The pages print no formula or
  * worked example for it; the tests pin it by closed forms, invariants and
@@ -297,6 +298,15 @@ static void attend_token_set(const uint16_t *q_row, const uint16_t *k_b,
                              double *logit)
 {
     const int G = Hq / Hkv;
+    if (n_keys == 0) {
+        /* Empty token set (only reachable with a caller-supplied selection
+         * that names no attendable token): the sum over no tokens, o = 0,
+         * and lse = ln 0 = -inf. */
+        for (int i = 0; i < Hq * D; ++i) o_row[i] = 0.0;
+        if (lse_row)
+            for (int h = 0; h < Hq; ++h) lse_row[h] = -INFINITY;
+        return;
+    }
     for (int h = 0; h < Hq; ++h) {
         const int g = h / G;
         double mx = -INFINITY;

@@ -260,6 +260,15 @@ def test_attn_golden(mode):
     np.testing.assert_allclose(lse[0], [_f(x) for x in g["expected_lse"]], rtol=1e-14)
 
 
+def test_attn_empty_token_set_is_zero():
+    """A selection naming no attendable token: the sum over no tokens (o = 0),
+    lse = ln 0 = -inf.  Blocks past the query's position and -1 entries."""
+    g, q, k, v = _attn_fixture()
+    o, lse = oracle.attn(q, k, v, 4, 1.0, sel=np.array([[-1, 5]], np.int32),
+                         q_pos0=np.array([1]))
+    assert (o == 0).all() and np.isneginf(lse).all()
+
+
 def _rand_qkv(rng, B, T, Hq, Hkv, D):
     q = _np_bf16(rng.standard_normal((B, T, Hq, D)))
     k = _np_bf16(rng.standard_normal((B, T, Hkv, D)))
