@@ -1,0 +1,618 @@
+#!/usr/bin/env python
+"""Benchmark of the QSA layer on B200 (one process per GPU).
+
+Default workload: QSA prefill of one 1M-token sequence (16 query heads, 2 KV
+heads, head dim 128, indexer 4 x 64, r = 4, token budget 2048) -- the context
+length the pages quote their attention speed-up at.  One step = the whole hot
+path: qsa_pool -> qsa_index_topk -> qsa_sparse_attn_prefill on inputs already
+in HBM.  With N GPUs every rank runs its own independent sequence (weak
+scaling, no data-path collective); the time is the max over ranks.
+
+The JSON line also carries: the dominant kernel's roofline fraction (CUDA
+events on the launch stream), an end-to-end figure through the C ABI with
+host buffers (H2D copies of the inputs and D2H of the output inside the timed
+region), the CPU oracle timed on a bounded sample of the same workload, the
+library's dense GQA attention on the same inputs (speed-up context), and
+secondary measurements (128K prefill, 64 x 256K decode).
+
+``--impl reference`` times the CPU oracle instead (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_long_10_b200 import synth  # noqa: E402
+
+METRIC = "QSA layer prefill tokens/s at 128K/1M; decode us/token at 256K; % roofline"
+L2_BYTES = 126 * 2**20
+BF = torch.bfloat16
+
+
+# ----------------------------------------------------------------- helpers --
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            sel = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None
+        except Exception:
+            sel = None
+        self.sel = sel
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="qsa_clocks_", suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if self.sel:
+            cmd += ["-i", self.sel]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.remove(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup(ngpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl" if torch.cuda.is_available() else "gloo",
+            timeout=datetime.timedelta(seconds=300))
+    if ngpus != world:
+        if rank == 0:
+            print(f"warning: --gpus {ngpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return rank, world, local
+
+
+def rank_seed(w: synth.Workload, rank: int) -> int:
+    """Each rank runs an independent sequence (weak scaling)."""
+    return w.seed + 7 * rank
+
+
+def aggregate_tokens_per_s(world: int, w: synth.Workload, ms_per_step_max: float) -> float:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's step time."""
+    return world * w.B * w.T / (ms_per_step_max / 1e3)
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------- algorithmic work models --
+
+def sparse_tokens_per_row(T: int, r: int, kb: int) -> np.ndarray:
+    """|S(t)| for p = t: 4 per selected complete block + the own block's
+    (t % r + 1) tokens; min(kb, c + 1) blocks."""
+    t = np.arange(T, dtype=np.int64)
+    c = t // r
+    nblk = np.minimum(kb, c + 1)
+    return r * (nblk - 1) + (t % r) + 1
+
+
+def prefill_work(w: synth.Workload) -> dict:
+    T, B = w.T, w.B
+    S = sparse_tokens_per_row(T, w.r, w.kb).astype(np.float64)
+    c = (np.arange(T) // w.r).astype(np.float64)
+    return {
+        "pool_bytes": B * (T * w.Di * 2 + (T // w.r) * w.Di * 2),
+        "index_flops": B * float(c.sum()) * 2 * w.Hi * w.Di,
+        "index_pairs": B * float(c.sum()),
+        "index_bytes": B * (T * w.Hi * w.Di * 2 + T * w.Hi * 4 + (T // w.r) * w.Di * 2
+                            + T * w.kb * 4),
+        "attn_bytes": B * (float(S.sum()) * w.Hkv * w.D * 2 * 2 + T * w.Hq * w.D * 2 * 2
+                           + T * w.kb * 4),
+        "attn_flops": B * float(S.sum()) * 4 * w.Hq * w.D,
+        "dense_flops": B * 4.0 * (T * (T + 1) / 2) * w.Hq * w.D,
+    }
+
+
+def decode_work(w: synth.Workload, seqlens) -> dict:
+    L = np.asarray(seqlens, np.int64)
+    c = (L - 1) // w.r
+    nblk = np.minimum(w.kb, c + 1)
+    S = w.r * (nblk - 1) + ((L - 1) % w.r) + 1
+    return {
+        "index_bytes": float((c * w.Di * 2).sum() + len(L) * (w.Hi * w.Di * 2 + w.kb * 4)),
+        "attn_bytes": float((S * w.Hkv * w.D * 2 * 2).sum() + len(L) * w.Hq * w.D * 4),
+        "dense_bytes": float((L * w.Hkv * w.D * 2 * 2).sum()),
+    }
+
+
+# ------------------------------------------------------------- GPU runners --
+
+class Prefill:
+    """Device buffers and one pass of the QSA prefill path for a workload."""
+
+    def __init__(self, qsa, w, x, device):
+        self.qsa, self.w, self.x = qsa, w, x
+        B, T = w.B, w.T
+        self.kp = torch.empty(B, T // w.r, w.Di, dtype=BF, device=device)
+        self.sel = torch.empty(B, T, w.kb, dtype=torch.int32, device=device)
+        self.o = torch.empty_like(x["q"])
+        self.ws = qsa.workspace(qsa.qsa_index_topk_workspace_size(
+            B, T, T // w.r, w.Hi, w.Di, w.r, w.budget), device)
+        self.stream = torch.cuda.current_stream(device)
+
+    def step(self, ev=None):
+        q, w, x = self.qsa, self.w, self.x
+        if ev:
+            ev[0].record(self.stream)
+        q.qsa_pool(x["k_idx"], self.kp, w.r, stream=self.stream)
+        if ev:
+            ev[1].record(self.stream)
+        q.qsa_index_topk(x["q_idx"], x["w"], self.kp, self.sel, self.ws, w.r, w.budget,
+                         stream=self.stream)
+        if ev:
+            ev[2].record(self.stream)
+        q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], self.sel, self.o, w.r, w.budget,
+                                  w.scale, stream=self.stream)
+        if ev:
+            ev[3].record(self.stream)
+
+    LAUNCHES = 3  # pool, index_topk, sparse_attn (the index counter reset is a memset)
+
+
+def events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def time_prefill(run: Prefill, steps: int, warmup: int, world: int, device, flush=None,
+                 clocks: Clocks | None = None):
+    for _ in range(warmup):
+        run.step()
+    torch.cuda.synchronize(device)
+    per = [events(4) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize(device)
+    if clocks:
+        clocks.start()
+    t0, t1 = events(2)
+    t0.record(run.stream)
+    for k in range(steps):
+        if flush is not None:
+            flush_l2(flush)
+        run.step(per[k])
+    t1.record(run.stream)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    total = t0.elapsed_time(t1)
+    kern = {"pool": 0.0, "index_topk": 0.0, "sparse_attn": 0.0}
+    for e in per:
+        kern["pool"] += e[0].elapsed_time(e[1])
+        kern["index_topk"] += e[1].elapsed_time(e[2])
+        kern["sparse_attn"] += e[2].elapsed_time(e[3])
+    kern = {k: v / steps for k, v in kern.items()}
+    return total, kern, clk
+
+
+def e2e_prefill(qsa, w, x, device, steps):
+    """Through the public API with host buffers: H2D of the step's inputs from
+    pinned memory, the three calls, D2H of the output, all inside the timing."""
+    names = ["q", "k", "v", "q_idx", "k_idx", "w"]
+    host = {n: torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True) for n in names}
+    for n in names:
+        host[n].copy_(x[n])
+    dev = {n: torch.empty_like(x[n]) for n in names}
+    run = Prefill(qsa, w, dev, device)
+    out_host = torch.empty(run.o.shape, dtype=BF, pin_memory=True)
+    s = run.stream
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        run.step()
+        out_host.copy_(run.o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(device)
+    a, b = events(2)
+    a.record(s)
+    for _ in range(steps):
+        one()
+    b.record(s)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    del host, dev, run, out_host
+    return ms, h2d, d2h
+
+
+def time_call(fn, stream, reps, warm=1, flush=None):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    evs = [events(2) for _ in range(reps)]
+    for e in evs:
+        if flush is not None:
+            flush_l2(flush)
+        e[0].record(stream)
+        fn()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    return sum(e[0].elapsed_time(e[1]) for e in evs) / reps
+
+
+def roof(achieved, peak, unit, bound, traffic=None):
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak if peak else None, "traffic": traffic}
+
+
+def kernel_report(w, kern_ms, peaks):
+    wk = prefill_work(w)
+    hbm = peaks["hbm_gbs"]
+    tf = peaks["bf16_tflops_sustained"]
+    rep = {}
+    for name, ms in kern_ms.items():
+        s = ms / 1e3
+        if name == "pool":
+            rep[name] = {"ms": ms, "GB/s": wk["pool_bytes"] / s / 1e9,
+                         "frac_hbm": wk["pool_bytes"] / s / 1e9 / hbm}
+        elif name == "index_topk":
+            rep[name] = {"ms": ms, "TFLOP/s": wk["index_flops"] / s / 1e12,
+                         "frac_tensor": wk["index_flops"] / s / 1e12 / tf,
+                         "pairs_per_s": wk["index_pairs"] / s}
+        elif name == "sparse_attn":
+            rep[name] = {"ms": ms, "GB/s": wk["attn_bytes"] / s / 1e9,
+                         "frac_hbm": wk["attn_bytes"] / s / 1e9 / hbm,
+                         "TFLOP/s": wk["attn_flops"] / s / 1e12,
+                         "frac_tensor": wk["attn_flops"] / s / 1e12 / tf}
+    return rep, wk
+
+
+def dominant_roofline(w, kern_ms, peaks, traffic=None):
+    wk = prefill_work(w)
+    name = max(kern_ms, key=kern_ms.get)
+    s = kern_ms[name] / 1e3
+    if name == "index_topk":
+        r = roof(wk["index_flops"] / s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s",
+                 "tensor", traffic)
+    elif name == "sparse_attn":
+        r = roof(wk["attn_bytes"] / s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm", traffic)
+    else:
+        r = roof(wk["pool_bytes"] / s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm", traffic)
+    r["kernel"] = name
+    r["peak_source"] = peaks["source"]
+    return r
+
+
+# ------------------------------------------------------- secondary workloads
+
+def extra_prefill(qsa, name, device, peaks, flush):
+    w = synth.WORKLOADS[name]
+    x = synth.make_prefill(w, device)
+    run = Prefill(qsa, w, x, device)
+    total, kern, _ = time_prefill(run, 5, 3, 1, device, flush=flush)
+    ms = total / 5
+    o = torch.empty_like(x["q"])
+    dense = time_call(lambda: qsa.qsa_dense_gqa_prefill(x["q"], x["k"], x["v"], o, w.scale),
+                      run.stream, 2, 1, flush)
+    rep, wk = kernel_report(w, kern, peaks)
+    out = {"ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3), "kernels": rep,
+           "dense_gqa_ms": dense,
+           "dense_gqa_tflops": wk["dense_flops"] / (dense / 1e3) / 1e12,
+           "dense_frac_tensor": wk["dense_flops"] / (dense / 1e3) / 1e12 / peaks["bf16_tflops"],
+           "speedup_vs_dense": dense / ms, "l2": "flushed between iterations"}
+    del x, run, o
+    torch.cuda.empty_cache()
+    return out
+
+
+def extra_decode(qsa, device, peaks, flush):
+    w = synth.WORKLOADS["decode-256k-b64"]
+    x = synth.make_decode(w, device)
+    B, L = w.B, w.T
+    kp = torch.empty(B, L // w.r, w.Di, dtype=BF, device=device)
+    qsa.qsa_pool(x["k_idx_cache"], kp, w.r)
+    sel = torch.empty(B, w.kb, dtype=torch.int32, device=device)
+    o = torch.empty_like(x["q"])
+    wsi = qsa.workspace(qsa.qsa_index_topk_decode_workspace_size(B, L // w.r, w.r, w.budget),
+                        device)
+    wsa = qsa.workspace(qsa.qsa_sparse_attn_decode_workspace_size(B, w.Hq, w.D, w.r, w.budget),
+                        device)
+    wsd = qsa.workspace(qsa.qsa_dense_gqa_decode_workspace_size(B, L, w.Hq, w.D), device)
+    s = torch.cuda.current_stream(device)
+    idx = lambda: qsa.qsa_index_topk_decode(x["q_idx"], x["w"], kp, x["seqlens"], sel, wsi,
+                                            w.r, w.budget, stream=s)
+    att = lambda: qsa.qsa_sparse_attn_decode(x["q"], x["k_cache"], x["v_cache"], x["seqlens"],
+                                             sel, o, wsa, w.r, w.budget, w.scale, stream=s)
+
+    def step():
+        idx()
+        att()
+
+    t_step = time_call(step, s, 20, 3, flush)
+    t_idx = time_call(idx, s, 20, 1, flush)
+    t_att = time_call(att, s, 20, 1, flush)
+    t_dense = time_call(lambda: qsa.qsa_dense_gqa_decode(x["q"], x["k_cache"], x["v_cache"],
+                                                         x["seqlens"], o, wsd, w.scale, stream=s),
+                        s, 5, 1, flush)
+    wk = decode_work(w, x["seqlens"].cpu().numpy())
+    hbm = peaks["hbm_gbs"]
+    out = {
+        "us_per_step": t_step * 1e3, "us_per_token": t_step * 1e3 / B, "batch": B,
+        "cache_len": L,
+        "kernels": {
+            "index_topk_decode": {"us": t_idx * 1e3,
+                                  "GB/s": wk["index_bytes"] / (t_idx / 1e3) / 1e9,
+                                  "frac_hbm": wk["index_bytes"] / (t_idx / 1e3) / 1e9 / hbm},
+            "sparse_attn_decode": {"us": t_att * 1e3,
+                                   "GB/s": wk["attn_bytes"] / (t_att / 1e3) / 1e9,
+                                   "frac_hbm": wk["attn_bytes"] / (t_att / 1e3) / 1e9 / hbm},
+        },
+        "step_frac_hbm": (wk["index_bytes"] + wk["attn_bytes"]) / (t_step / 1e3) / 1e9 / hbm,
+        "dense_gqa_us": t_dense * 1e3,
+        "dense_frac_hbm": wk["dense_bytes"] / (t_dense / 1e3) / 1e9 / hbm,
+        "speedup_vs_dense": t_dense / t_step, "l2": "flushed between iterations",
+        "launches_per_step": 4,
+    }
+    del x, kp
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample(w: synth.Workload, x: dict, n_rows: int, seed: int, threads: int | None = None):
+    """Time the CPU oracle on stratified query rows of the workload.
+
+    Rows are drawn one per equal-width stratum of [0, T) so that their mean
+    cost estimates the mean over all rows; pooling is timed over the whole
+    sequence and charged per token.  Returns (tokens/s, seconds, rows)."""
+    import oracle  # test/baseline infrastructure only
+    if threads:
+        oracle.set_num_threads(threads)
+    host = {n: synth.bf16_bits(x[n]) for n in ("q", "k", "v", "q_idx", "k_idx")}
+    wt = x["w"].cpu().numpy()
+    t0 = time.perf_counter()
+    kp = oracle.pool(host["k_idx"], w.r)
+    t_pool = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    edges = np.linspace(0, w.T, n_rows + 1).astype(np.int64)
+    rows = np.array([rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))
+                     for i in range(n_rows)], np.int64)
+    t0 = time.perf_counter()
+    sel, _, _, _ = oracle.index_topk(host["q_idx"], wt, kp, w.r, w.budget, rows=rows)
+    oracle.attn(host["q"], host["k"], host["v"], w.r, w.scale, sel=sel, rows=rows)
+    t_rows = time.perf_counter() - t0
+    per_token = t_rows / n_rows + t_pool / (w.B * w.T)
+    return 1.0 / per_token, t_rows + t_pool, rows.size
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# -------------------------------------------------------------------- main --
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    x = synth.make_prefill(w, device)
+    import oracle
+    cores = oracle.num_threads()
+    n_rows = args.ref_rows
+    for k in range(args.warmup):
+        oracle_sample(w, x, max(8, n_rows // 4), seed=1000 + k)
+    vals, secs = [], []
+    for k in range(args.steps):
+        v, s, _ = oracle_sample(w, x, n_rows, seed=k)
+        vals.append(v)
+        secs.append(s)
+    value = len(vals) / sum(1.0 / v for v in vals)  # tokens over total time
+    sample = (f"{n_rows} stratified query rows of the {w.name} workload per step "
+              f"(index top-k + attention per row, pooling charged per token), "
+              f"rows/s extrapolated to tokens/s")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(secs) / len(secs), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, "oracle on a stratified row sample"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, l2):
+    return {"workload": w.name, "batch": w.B, "seq_len": w.T, "q_heads": w.Hq,
+            "kv_heads": w.Hkv, "head_dim": w.D, "indexer_heads": w.Hi, "indexer_dim": w.Di,
+            "block": w.r, "token_budget": w.budget, "seed": w.seed, "l2": l2}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
+    ap.add_argument("--workload", default="prefill-1m",
+                    choices=[n for n, w in synth.WORKLOADS.items() if w.kind == "prefill"])
+    ap.add_argument("--no-extra", action="store_true", help="skip 128K and decode lines")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense GQA ratio run")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    import block_sparse_long_10_b200 as qsa
+    qsa.load()  # fails loudly if the CUDA library is missing
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    w = synth.WORKLOADS[args.workload]
+    seed = rank_seed(w, rank)
+    x = synth.make_prefill(w, device, seed=seed)
+    in_bytes = sum(x[n].numel() * x[n].element_size()
+                   for n in ("q", "k", "v", "q_idx", "k_idx", "w"))
+    run = Prefill(qsa, w, x, device)
+    flush = None
+    if in_bytes < 4 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    clocks = Clocks(local)
+    total_ms, kern, clk = time_prefill(run, args.steps, args.warmup, world, device,
+                                       flush=flush, clocks=clocks)
+    total_ms = max_over_ranks(total_ms, world, device)
+    ms_step = total_ms / args.steps
+    value = aggregate_tokens_per_s(world, w, ms_step)
+    kern_rep, wk = kernel_report(w, kern, peaks)
+    roofline = dominant_roofline(w, kern, peaks)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": config_of(w, "flushed between steps" if flush is not None else
+                            f"inputs larger than L2 ({in_bytes / 1e9:.1f} GB per step)"),
+        "roofline": roofline, "kernels": kern_rep,
+        "gpu_launches": Prefill.LAUNCHES * args.steps,
+        "clocks": clk,
+    }
+    barrier(world)
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_prefill(qsa, w, x, device, min(args.steps, 5))
+        e2e_ms = max_over_ranks(e2e_ms, world, device)
+        line["e2e"] = {"value": world * w.B * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e2e_ms}
+    barrier(world)
+    if rank == 0:
+        if not args.no_dense:
+            o = torch.empty_like(x["q"])
+            if w.T >= 2**19:  # load the kernel on a short prefix first
+                qsa.qsa_dense_gqa_prefill(x["q"][:, :4096].contiguous(),
+                                          x["k"][:, :4096].contiguous(),
+                                          x["v"][:, :4096].contiguous(),
+                                          o[:, :4096].contiguous(), w.scale)
+            d_ms = time_call(lambda: qsa.qsa_dense_gqa_prefill(x["q"], x["k"], x["v"], o, w.scale),
+                             run.stream, 1, 0 if w.T >= 2**19 else 1, flush)
+            line["dense_gqa"] = {"ms": d_ms,
+                                 "tflops": wk["dense_flops"] / (d_ms / 1e3) / 1e12,
+                                 "frac_tensor": wk["dense_flops"] / (d_ms / 1e3) / 1e12
+                                 / peaks["bf16_tflops"],
+                                 "speedup_qsa_vs_dense": d_ms / ms_step}
+            del o
+        if not args.no_cpu and world == 1:
+            v, secs, n = oracle_sample(w, x, args.cpu_rows, seed=12345)
+            line["cpu_baseline"] = {
+                "value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                "sample": f"{n} stratified query rows of {w.name} (index top-k + attention "
+                          f"per row) plus pooling of the whole sequence, {secs:.1f} s wall; "
+                          f"rows/s extrapolated to tokens/s"}
+        if not args.no_extra:
+            del run
+            torch.cuda.empty_cache()
+            fl = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+            line["extra"] = {}
+            if w.name != "prefill-128k":
+                line["extra"]["prefill-128k"] = extra_prefill(qsa, "prefill-128k", device, peaks, fl)
+            line["extra"]["decode-256k-b64"] = extra_decode(qsa, device, peaks, fl)
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

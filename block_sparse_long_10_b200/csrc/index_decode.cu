@@ -33,9 +33,10 @@ QSA_DEVICE uint64_t make_key(float s, int j) {
 }
 
 // Block-wide radix select: the K-th largest of n unique keys (1 <= K <= n).
-// `hist` holds 256 counters, `sh` two ints; all threads must call.
+// `hist` holds 256 counters, `sh` four ints, `red` one u64 per warp; all threads
+// must call.
 QSA_DEVICE uint64_t block_kth_largest(const uint64_t *keys, int n, int K, uint32_t *hist,
-                                      int *sh) {
+                                      int *sh, uint64_t *red) {
     const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31;
     uint64_t prefix = 0;
     int want = K;
@@ -75,12 +76,34 @@ QSA_DEVICE uint64_t block_kth_largest(const uint64_t *keys, int n, int K, uint32
             if (found >= 0) {
                 sh[0] = found;
                 sh[1] = nw;
+                sh[3] = (int)local[found - lane * 8];
             }
         }
         __syncthreads();
         prefix |= (uint64_t)(uint32_t)sh[0] << shift;
         want = sh[1];
+        const int bucket = sh[3];
         __syncthreads();
+        if (shift > 0 && bucket == want) {
+            // every key of this bucket is kept: the K-th largest is its minimum
+            const uint64_t m = ~0ull << shift;
+            uint64_t mn = ~0ull;
+            for (int i = tid; i < n; i += nth) {
+                const uint64_t k = keys[i];
+                if ((k & m) == prefix && k < mn) mn = k;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const uint64_t o = __shfl_xor_sync(0xffffffffu, mn, off);
+                mn = o < mn ? o : mn;
+            }
+            if (lane == 0) red[tid >> 5] = mn;
+            __syncthreads();
+            mn = ~0ull;
+            for (int i = 0; i < nth / 32; ++i) mn = red[i] < mn ? red[i] : mn;
+            __syncthreads();
+            return mn;
+        }
     }
     return prefix;
 }
@@ -97,6 +120,7 @@ __global__ void __launch_bounds__(THREADS, 3)
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     __shared__ uint32_t hist[256];
     __shared__ int sh[4];
+    __shared__ uint64_t red[THREADS / 32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int lr = lane >> 2, lc = lane & 3;
     const int b = blockIdx.x / nsplit, split = blockIdx.x % nsplit;
@@ -188,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 3)
         if (tid == 0) part_cnt[b * nsplit + split] = n;
         return;
     }
-    const uint64_t kth = block_kth_largest(keys, n, K, hist, sh);
+    const uint64_t kth = block_kth_largest(keys, n, K, hist, sh, red);
     if (tid == 0) sh[2] = 0;
     __syncthreads();
     for (int i = tid; i < n; i += THREADS) {
@@ -208,6 +232,7 @@ __global__ void __launch_bounds__(MERGE_THREADS)
     uint64_t *sorted = keys + cap_n;                        // [<= 1024] kept keys
     __shared__ uint32_t hist[256];
     __shared__ int sh[4];
+    __shared__ uint64_t red[MERGE_THREADS / 32];
     const int tid = threadIdx.x;
     const int b = blockIdx.x;
     const int K = kb - 1;
@@ -224,7 +249,7 @@ __global__ void __launch_bounds__(MERGE_THREADS)
     }
     __syncthreads();
     if (n > K) {
-        const uint64_t kth = block_kth_largest(keys, n, K, hist, sh);
+        const uint64_t kth = block_kth_largest(keys, n, K, hist, sh, red);
         if (tid == 0) sh[2] = 0;
         __syncthreads();
         for (int i = tid; i < n; i += MERGE_THREADS) {

@@ -102,10 +102,26 @@ QSA_DEVICE uint64_t warp_kth_largest(const uint64_t *buf, int n, int K, uint32_t
         }
         const uint32_t ball = __ballot_sync(0xffffffffu, found >= 0);
         const int src = __ffs(ball) - 1;
+        const uint32_t bucket = __shfl_sync(0xffffffffu, found >= 0 ? hist[found] : 0u, src);
         found = __shfl_sync(0xffffffffu, found, src);
         want = __shfl_sync(0xffffffffu, new_want, src);
         prefix |= (uint64_t)(uint32_t)found << shift;
         __syncwarp();
+        if (shift > 0 && (int)bucket == want) {
+            // every key of this bucket is kept: the K-th largest is its minimum
+            const uint64_t m = ~0ull << shift;
+            uint64_t mn = ~0ull;
+            for (int i = lane; i < n; i += 32) {
+                const uint64_t k = buf[i];
+                if ((k & m) == prefix && k < mn) mn = k;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const uint64_t o = __shfl_xor_sync(0xffffffffu, mn, off);
+                mn = o < mn ? o : mn;
+            }
+            return mn;
+        }
     }
     return prefix;
 }
