@@ -24,7 +24,8 @@ __all__ = [
     "qsa_pool", "qsa_index_topk", "qsa_index_topk_workspace_size",
     "qsa_index_topk_decode", "qsa_index_topk_decode_workspace_size",
     "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode",
-    "qsa_sparse_attn_decode_workspace_size", "qsa_dense_gqa_prefill",
+    "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode_noalloc",
+    "qsa_dense_gqa_prefill",
     "qsa_dense_gqa_decode", "qsa_dense_gqa_decode_workspace_size",
     "qsa_check_device_status", "qsa_status_string", "qsa_version",
 ]
@@ -65,6 +66,8 @@ _SIGS = {
     "qsa_sparse_attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "qsa_sparse_attn_decode": (_I, [_VP, _VP, _VP, _VP, _I64, _VP, _I, _I, _I,
                                     _I, _I, _I, _F, _VP, _VP, _VP, _SZ, _VP]),
+    "qsa_sparse_attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _I64, _VP, _I, _I, _I,
+                                            _I, _I, _I, _F, _VP, _VP, _VP]),
     "qsa_dense_gqa_prefill": (_I, [_VP, _VP, _VP, _I, _I64, _I, _I, _I, _F, _VP,
                                    _VP, _VP]),
     "qsa_dense_gqa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I]),
@@ -232,6 +235,27 @@ def qsa_sparse_attn_decode(q, k_cache, v_cache, seqlens, sel, o, ws, r=4, budget
     scale = D ** -0.5 if scale is None else scale
     _call("qsa_sparse_attn_decode", _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), L,
           _ptr(sel), B, Hq, Hkv, D, r, budget, scale, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+          _stream(stream, q.device))
+
+
+def qsa_sparse_attn_decode_noalloc(q, k_cache, v_cache, seqlens, sel, o, r=4, budget=2048,
+                                   scale=None, lse=None, stream=None):
+    """qsa_sparse_attn_decode without a workspace, for callers that cannot
+    allocate device memory where they run the step: the library keeps the
+    split partials in its own fixed 8 MiB device array (shared by all calls on
+    a device; concurrent calls race).  Too large a batch raises QSAError."""
+    _need(q, _BF, "q", 3)
+    _need(k_cache, _BF, "k_cache", 4)
+    _need(v_cache, _BF, "v_cache", 4)
+    _need(o, _BF, "o", 3)
+    _need(seqlens, _I32, "seqlens", 1)
+    _need(sel, _I32, "sel", 2)
+    _need(lse, _F32, "lse", 2)
+    B, Hq, D = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    scale = D ** -0.5 if scale is None else scale
+    _call("qsa_sparse_attn_decode_noalloc", _ptr(q), _ptr(k_cache), _ptr(v_cache),
+          _ptr(seqlens), L, _ptr(sel), B, Hq, Hkv, D, r, budget, scale, _ptr(o), _ptr(lse),
           _stream(stream, q.device))
 
 

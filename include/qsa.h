@@ -177,6 +177,38 @@ QSA_API qsa_status_t qsa_sparse_attn_decode(const qsa_bf16_t *q, const qsa_bf16_
                                     size_t ws_bytes, void *stream);
 
 /*
+ * Sparse decode attention without a caller workspace.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory where they run a decode step (for example an engine plugin
+ * whose enqueue must not allocate, or a server whose device memory budget is
+ * fixed at start-up) and so cannot provide the workspace that
+ * qsa_sparse_attn_decode takes.
+ *
+ * Same arguments, definition and outputs as qsa_sparse_attn_decode, minus the
+ * workspace.  The split partials live in one library-owned device array of
+ * QSA_NOALLOC_SCRATCH_BYTES (8 MiB) per GPU, held from library load until
+ * process exit; the call allocates nothing.  Requirements and behaviour:
+ *   - B * nsplit * Hq * (D + 2) * 4 bytes must fit in the array, with
+ *     nsplit = min(ceil(512 / B), max(1, kb / 16)); larger problems return
+ *     QSA_ERR_WORKSPACE before anything is enqueued (the 64 x 16-head x 128
+ *     decode batch needs 4.3 MB).
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array: calls that may run at the same
+ *     time on the GPU (other streams, other threads) race and must be
+ *     serialised by the caller.  Nothing in the array needs to start at zero:
+ *     every partial a call reads is written by that call first.
+ *   - Out-of-range seqlens are handled as in qsa_sparse_attn_decode but not
+ *     recorded (there is no workspace status word).
+ */
+#define QSA_NOALLOC_SCRATCH_BYTES (8u << 20)
+QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
+    const qsa_bf16_t *q, const qsa_bf16_t *k_cache, const qsa_bf16_t *v_cache,
+    const int32_t *seqlens, int64_t L_max, const int32_t *sel, int B, int Hq, int Hkv, int D,
+    int r, int budget, float scale, qsa_bf16_t *o, float *lse, void *stream);
+
+/*
  * Dense causal GQA attention, prefill: every query t attends to all tokens
  * u <= t (the full-attention layer QSA replaces; speed-up baseline).
  *   q [B, T, Hq, D], k, v [B, T, Hkv, D], o [B, T, Hq, D] bf16;
