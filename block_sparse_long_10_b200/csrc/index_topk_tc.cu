@@ -1,0 +1,624 @@
+// Lightweight MQA indexer on tcgen05: fused block scores + exact top-k.
+//
+// "用125亿分之6的参数，打平3970亿的旗舰模型", section
+// "稀疏注意力：给检索建索引，也得先学会省纸": a lightweight MQA indexer (several
+// query heads, one shared pooled key head) scores every micro-block and the
+// highest-scoring blocks are kept, following DSA's lightweight indexer;
+// "On the Design of Qwen3.8-Next Architecture" (token-mixing paragraph):
+// indexing O(n^2 / r), token budget 2048.
+//
+//   s(t, j) = sum_h w[t, h] * max(0, q_idx[t, h, :] . Kp[j, :])   (fp32)
+//   keep the kb - 1 best j < floor(p / r) by (s desc, j asc) + own block.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: the CTA's query tile (NCOL (query, head) rows,
+//               double-buffered) and a 4-stage ring of 128-block pooled-key
+//               tiles, 128/64-byte swizzled;
+//   warp 1      TMEM owner and MMA issuer: per pooled-key tile one thread
+//               issues D[128 blocks, NCOL columns] = Kp_tile x Q_tile^T as
+//               Di/16 tcgen05.mma (bf16 in, fp32 in TMEM), double-buffered;
+//   warps 2-17  epilogue: TMEM lane = block, so each thread reads one block's
+//               scores for a quarter of the columns (32x32b loads) and forms
+//               the ReLU-weighted head sum in registers.
+// Each query tile is swept twice (the pooled keys stay in L2):
+//   pass 1  every thread keeps, per query, the maximum score of its block
+//           lane over groups of R consecutive tiles (at most 8 groups, so at
+//           most 1024 group maxima per query).  The group maxima are distinct
+//           candidates, so the (kb-1)-th largest of them, theta, is a lower
+//           bound of the true (kb-1)-th best score; with ~1024 groups it is
+//           tight (a few hundred survivors beyond kb - 1 on random data).
+//   pass 2  the same scores, recomputed bit for bit, are filtered by
+//           s >= theta and appended (64-bit key: order-preserving score bits
+//           above the complemented block index) to the query's list in the
+//           workspace.  Every top-(kb-1) candidate has s >= theta.
+// Finalisation (per query): exact radix select of the list's kb - 1 best
+// keys in shared memory, stable radix sort by block id, own block appended.
+// A list that would overflow (only with heavily tied scores) is cut to its
+// kb - 1 best keys on the spot and the filter becomes strict, which is exact
+// because blocks are swept in ascending order.  Scores never reach HBM.
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "qsa_common.cuh"
+#include "qsa_launch.h"
+#include "sm100.cuh"
+#include "topk_warp.cuh"
+
+namespace qsa {
+namespace itc {
+
+constexpr int MB = 128;          // pooled blocks per tile = MMA M = TMEM lanes
+constexpr int STAGES = 4;
+constexpr int EPI_WARPS = 16;    // 4 per TMEM lane quarter
+constexpr int SEL_WARPS = 8;     // epilogue warps that also run the selections
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr int CAP = 2048;        // candidate-list capacity per query (workspace)
+constexpr int SELBUF = 1024;     // per selecting warp, u64 keys in shared memory
+constexpr int MAX_GROUPS = 8;    // group maxima per block lane and query
+constexpr int MAX_KEEP = 511;
+constexpr int MAX_GRID = 160;
+
+template <int HI, int DI>
+struct L {
+    static constexpr int NCOL = HI == 1 ? 128 : 256;  // MMA N
+    static constexpr int QT = NCOL / HI;              // queries per tile
+    static constexpr int QPT = NCOL / 4 / HI;         // queries per epilogue thread
+    static constexpr int ROWB = DI * 2;               // 64 or 128 bytes (= swizzle width)
+    static constexpr int KP_TILE = MB * ROWB;
+    static constexpr int Q_TILE = NCOL * ROWB;
+    static constexpr int OFF_KP = 0;
+    static constexpr int OFF_Q = OFF_KP + STAGES * KP_TILE;
+    static constexpr int OFF_BUF = OFF_Q + 2 * Q_TILE;
+    static constexpr int OFF_HIST = OFF_BUF + SEL_WARPS * SELBUF * 8;
+    static constexpr int OFF_W = OFF_HIST + SEL_WARPS * 256 * 4;
+    static constexpr int OFF_THR = OFF_W + QT * 16;
+    static constexpr int OFF_C = OFF_THR + QT * 4;
+    static constexpr int OFF_CNT = OFF_C + QT * 4;
+    static constexpr int OFF_BAR = OFF_CNT + QT * 4;
+    static constexpr int NBAR = 2 * STAGES + 9;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int BYTES = OFF_MISC + 64;
+    static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1 KiB
+};
+
+struct Args {
+    const float *w;
+    const int64_t *q_pos0;
+    int B;
+    int64_t Tq, n_blocks;
+    int kb;
+    int32_t *sel;
+    float *sel_score;
+    uint8_t *ws;
+    int n_qt, total_tiles;
+    uint32_t wait_limit;
+    int grid;
+};
+
+QSA_DEVICE void epi_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(EPI_WARPS * 32) : "memory"); }
+
+QSA_DEVICE int64_t causal_blocks(int64_t pos, int64_t n_blocks, void *status) {
+    if (pos < 0) return 0;
+    int64_t c = pos / 4;
+    if (c > n_blocks) {
+        record_status(status, QSA_ERR_DEVICE);
+        c = n_blocks;
+    }
+    return c;
+}
+
+// Per query tile geometry, identical in every role.
+struct TileGeo {
+    int b;
+    int64_t t0, pb, c_min, c_max;
+    int n_kt, R;
+};
+
+template <int QT>
+QSA_DEVICE TileGeo tile_geo(const Args &a, int tile) {
+    TileGeo g;
+    g.b = tile % a.B;
+    const int qt = a.n_qt - 1 - tile / a.B;  // longest query tiles first
+    g.t0 = (int64_t)qt * QT;
+    g.pb = a.q_pos0 ? a.q_pos0[g.b] : 0;
+    const int64_t t_last = (g.t0 + QT < a.Tq ? g.t0 + QT : a.Tq) - 1;
+    g.c_max = causal_blocks(g.pb + t_last, a.n_blocks, nullptr);
+    g.c_min = causal_blocks(g.pb + g.t0, a.n_blocks, nullptr);
+    g.n_kt = (int)((g.c_max + MB - 1) / MB);
+    g.R = (g.n_kt + MAX_GROUPS - 1) / MAX_GROUPS;
+    if (g.R < 1) g.R = 1;
+    return g;
+}
+
+template <int HI>
+QSA_DEVICE float score_of(const uint32_t *v, const float4 wq) {
+    const float wa[4] = {wq.x, wq.y, wq.z, wq.w};
+    float s = 0.f;
+#pragma unroll
+    for (int h = 0; h < HI; ++h) s = fmaf(wa[h], fmaxf(__uint_as_float(v[h]), 0.f), s);
+    return s;
+}
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(THREADS, 1)
+    idx_tc_kernel(const __grid_constant__ CUtensorMap tm_kp,
+                  const __grid_constant__ CUtensorMap tm_q, const Args a) {
+    using Lx = L<HI, DI>;
+    constexpr int NCOL = Lx::NCOL;
+    constexpr int QT = Lx::QT;
+    constexpr int QPT = Lx::QPT;
+    constexpr int KSTEPS = DI / 16;
+    constexpr uint32_t IDESC = sm100::idesc_bf16_f32(MB, NCOL);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    float4 *s_w = reinterpret_cast<float4 *>(sm + Lx::OFF_W);
+    float *s_thr = reinterpret_cast<float *>(sm + Lx::OFF_THR);
+    int *s_c = reinterpret_cast<int *>(sm + Lx::OFF_C);
+    int *s_cnt = reinterpret_cast<int *>(sm + Lx::OFF_CNT);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Lx::OFF_BAR);
+    uint64_t *full = bar, *empty = bar + STAGES;
+    uint64_t *tfull = bar + 2 * STAGES, *tempty = tfull + 2;
+    uint64_t *qfull = tfull + 4, *qempty = tfull + 6;
+    uint64_t *mma_done = tfull + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lx::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lx::OFF_MISC + 8);
+    volatile int *overflow = reinterpret_cast<volatile int *>(sm + Lx::OFF_MISC + 16);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int K = a.kb - 1;
+    // workspace: candidate lists, then group maxima, per CTA
+    uint64_t *lists = reinterpret_cast<uint64_t *>(a.ws + kWsHeader) + (size_t)blockIdx.x * QT * CAP;
+    uint32_t *gmax_g = reinterpret_cast<uint32_t *>(reinterpret_cast<uint64_t *>(a.ws + kWsHeader) +
+                                                    (size_t)a.grid * QT * CAP) +
+                       (size_t)blockIdx.x * QT * (MAX_GROUPS * MB);
+
+    if (tid == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            sm100::mbar_init(&full[i], 1);
+            sm100::mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            sm100::mbar_init(&tfull[i], 1);
+            sm100::mbar_init(&tempty[i], EPI_WARPS);
+            sm100::mbar_init(&qfull[i], 1);
+            sm100::mbar_init(&qempty[i], 1);
+        }
+        sm100::mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        *overflow = 0;
+        sm100::fence_mbar_init();
+    }
+    if (warp == 1) sm100::tmem_alloc(tmem_slot, 2 * NCOL);
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer --
+        if (lane == 0) {
+            sm100::prefetch_tensormap(&tm_kp);
+            sm100::prefetch_tensormap(&tm_q);
+            uint32_t it = 0;
+            int last_kp[STAGES], last_q[2] = {-1, -1};  // most recent load per buffer
+            for (int s2 = 0; s2 < STAGES; ++s2) last_kp[s2] = -1;
+            for (int i = 0;; ++i) {
+                const int tile = blockIdx.x + i * gridDim.x;
+                if (tile >= a.total_tiles) break;
+                const TileGeo g = tile_geo<QT>(a, tile);
+                const int qb = i & 1;
+                if (sm100::mbar_wait(&qempty[qb], ((i >> 1) & 1) ^ 1, abort_flag, a.wait_limit,
+                                     a.ws)) {
+                    sm100::mbar_arrive_expect_tx(&qfull[qb], Lx::Q_TILE);
+                    sm100::tma_load_2d(sm + Lx::OFF_Q + qb * Lx::Q_TILE, &tm_q, 0,
+                                       (int32_t)(((int64_t)g.b * a.Tq + g.t0) * HI), &qfull[qb]);
+                    last_q[qb] = i;
+                }
+                for (int pass = 0; pass < 2; ++pass)
+                    for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
+                        const int s = it % STAGES;
+                        if (!sm100::mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag,
+                                              a.wait_limit, a.ws))
+                            continue;
+                        sm100::mbar_arrive_expect_tx(&full[s], Lx::KP_TILE);
+                        sm100::tma_load_2d(sm + Lx::OFF_KP + s * Lx::KP_TILE, &tm_kp, 0,
+                                           (int32_t)((int64_t)g.b * a.n_blocks + (int64_t)kt * MB),
+                                           &full[s]);
+                        last_kp[s] = (int)it;
+                    }
+            }
+            if (*abort_flag) {
+                // let this CTA's own copies in flight land before it exits (bounded)
+                for (int s2 = 0; s2 < STAGES; ++s2)
+                    if (last_kp[s2] >= 0)
+                        for (uint32_t n = 0; n < (1u << 20); ++n)
+                            if (sm100::mbar_try_wait(&full[s2], (last_kp[s2] / STAGES) & 1)) break;
+                for (int qb = 0; qb < 2; ++qb)
+                    if (last_q[qb] >= 0)
+                        for (uint32_t n = 0; n < (1u << 20); ++n)
+                            if (sm100::mbar_try_wait(&qfull[qb], (last_q[qb] >> 1) & 1)) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int i = 0;; ++i) {
+                const int tile = blockIdx.x + i * gridDim.x;
+                if (tile >= a.total_tiles) break;
+                const TileGeo g = tile_geo<QT>(a, tile);
+                const int qb = i & 1;
+                const bool q_ok =
+                    sm100::mbar_wait(&qfull[qb], (i >> 1) & 1, abort_flag, a.wait_limit, a.ws);
+                sm100::tc_fence_after();
+                const uint32_t b_base = smem_u32(sm + Lx::OFF_Q + qb * Lx::Q_TILE);
+                for (int pass = 0; pass < 2; ++pass)
+                    for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
+                        const int s = it % STAGES;
+                        const int tb = it & 1;
+                        const bool ok = q_ok &&
+                                        sm100::mbar_wait(&full[s], (it / STAGES) & 1, abort_flag,
+                                                         a.wait_limit, a.ws) &&
+                                        sm100::mbar_wait(&tempty[tb], ((it >> 1) & 1) ^ 1,
+                                                         abort_flag, a.wait_limit, a.ws);
+                        if (!ok) continue;
+                        sm100::tc_fence_after();
+                        const uint32_t a_base = smem_u32(sm + Lx::OFF_KP + s * Lx::KP_TILE);
+#pragma unroll
+                        for (int k = 0; k < KSTEPS; ++k)
+                            sm100::mma_bf16(tmem_base + tb * NCOL,
+                                            sm100::smem_desc_kmajor(a_base + k * 32, Lx::ROWB),
+                                            sm100::smem_desc_kmajor(b_base + k * 32, Lx::ROWB),
+                                            IDESC, k > 0);
+                        sm100::mma_commit(&empty[s]);
+                        sm100::mma_commit(&tfull[tb]);
+                    }
+                if (q_ok) sm100::mma_commit(&qempty[qb]);
+            }
+            // every MMA this thread issued has retired before TMEM is freed (bounded)
+            sm100::mma_commit(mma_done);
+            for (uint32_t n = 0; n < (1u << 22); ++n)
+                if (sm100::mbar_try_wait(mma_done, 0)) break;
+        }
+    } else {
+        // ------------------------------------------------------ epilogue --
+        const int e = warp - 2;                 // 0..15
+        const int etid = tid - 64;
+        const int lq = warp & 3;                // TMEM lane quarter this warp may read
+        const int cq = e >> 2;                  // column quarter
+        const int q0 = cq * QPT;                // first query of this thread
+        const int p = lq * 32 + lane;           // block position within the tile
+        const bool selw = e < SEL_WARPS;
+        uint32_t *hist = reinterpret_cast<uint32_t *>(sm + Lx::OFF_HIST) + (selw ? e : 0) * 256;
+        uint64_t *buf = reinterpret_cast<uint64_t *>(sm + Lx::OFF_BUF) + (size_t)(selw ? e : 0) * SELBUF;
+        int sort_passes = 1;
+        while (sort_passes < 4 && (a.n_blocks >> (8 * sort_passes)) > 0) ++sort_passes;
+        uint32_t it = 0;
+        for (int i = 0;; ++i) {
+            const int tile = blockIdx.x + i * gridDim.x;
+            if (tile >= a.total_tiles) break;
+            const TileGeo g = tile_geo<QT>(a, tile);
+            const int n_groups = (g.n_kt + g.R - 1) / g.R;
+
+            for (int q = etid; q < QT; q += EPI_WARPS * 32) {
+                const int64_t t = g.t0 + q;
+                float wv[4] = {0.f, 0.f, 0.f, 0.f};
+                int c = 0;
+                if (t < a.Tq) {
+                    c = (int)causal_blocks(g.pb + t, a.n_blocks, a.ws);
+                    const float *wr = a.w + ((int64_t)g.b * a.Tq + t) * HI;
+#pragma unroll
+                    for (int h = 0; h < HI; ++h) wv[h] = wr[h];
+                }
+                s_w[q] = make_float4(wv[0], wv[1], wv[2], wv[3]);
+                s_c[q] = c;
+                s_cnt[q] = 0;
+            }
+            epi_sync();
+
+            // ---- pass 1: group maxima -----------------------------------
+            float gm[QPT];
+#pragma unroll
+            for (int x = 0; x < QPT; ++x) gm[x] = -INFINITY;
+            for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
+                const int tb = it & 1;
+                sm100::mbar_wait(&tfull[tb], (it >> 1) & 1, abort_flag, a.wait_limit, a.ws);
+                sm100::tc_fence_after();
+                const int j = kt * MB + p;
+                const bool tail = (int64_t)kt * MB + MB > g.c_min;
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
+#pragma unroll
+                for (int ch = 0; ch < NCOL / 4 / 32; ++ch) {
+                    uint32_t v[32];
+                    sm100::tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+                    for (int qq = 0; qq < 32 / HI; ++qq) {
+                        const int x = ch * (32 / HI) + qq;
+                        const float s = score_of<HI>(v + qq * HI, s_w[q0 + x]);
+                        if (!tail || j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], s);
+                    }
+                }
+                sm100::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(&tempty[tb]);
+                if ((kt + 1) % g.R == 0 || kt + 1 == g.n_kt) {
+                    const int grp = kt / g.R;
+#pragma unroll
+                    for (int x = 0; x < QPT; ++x) {
+                        gmax_g[(size_t)(q0 + x) * (MAX_GROUPS * MB) + grp * MB + p] = score_key(gm[x]);
+                        gm[x] = -INFINITY;
+                    }
+                }
+            }
+            epi_sync();
+
+            // ---- theta: the (kb-1)-th largest group maximum --------------
+            if (selw) {
+#pragma unroll 1
+                for (int q = e; q < QT; q += SEL_WARPS) {
+                    float th = K > 0 ? -INFINITY : INFINITY;
+                    const int G = n_groups * MB;
+                    if (K > 0 && G >= K && g.t0 + q < a.Tq) {
+                        const uint32_t *src = gmax_g + (size_t)q * (MAX_GROUPS * MB);
+                        for (int x = lane; x < G; x += 32)
+                            buf[x] = ((uint64_t)src[x] << 32) | (uint32_t)x;
+                        __syncwarp();
+                        const uint64_t kth = idx::warp_kth_largest(buf, G, K, hist, lane);
+                        th = key_score((uint32_t)(kth >> 32));
+                    }
+                    if (g.t0 + q >= a.Tq) th = INFINITY;   // padding queries keep nothing
+                    if (lane == 0) s_thr[q] = th;
+                    __syncwarp();
+                }
+            }
+            epi_sync();
+
+            // ---- pass 2: keep every candidate with s >= theta ------------
+            float th[QPT];
+#pragma unroll
+            for (int x = 0; x < QPT; ++x) th[x] = s_thr[q0 + x];
+            for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
+                const int tb = it & 1;
+                sm100::mbar_wait(&tfull[tb], (it >> 1) & 1, abort_flag, a.wait_limit, a.ws);
+                sm100::tc_fence_after();
+                const int j = kt * MB + p;
+                const bool tail = (int64_t)kt * MB + MB > g.c_min;
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
+#pragma unroll
+                for (int ch = 0; ch < NCOL / 4 / 32; ++ch) {
+                    uint32_t v[32];
+                    sm100::tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+                    for (int qq = 0; qq < 32 / HI; ++qq) {
+                        const int x = ch * (32 / HI) + qq;
+                        const float s = score_of<HI>(v + qq * HI, s_w[q0 + x]);
+                        if (s >= th[x] && (!tail || j < s_c[q0 + x])) {
+                            const int pos = atomicAdd(&s_cnt[q0 + x], 1);
+                            if (pos < CAP)
+                                lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(s, j);
+                            if (pos == CAP - 2 * MB) *overflow = 1;
+                        }
+                    }
+                }
+                sm100::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(&tempty[tb]);
+                epi_sync();
+                if (*overflow) {  // uniform: read after the barrier, set only before it
+                    if (selw) {
+#pragma unroll 1
+                        for (int q = e; q < QT; q += SEL_WARPS) {
+                            const int n = s_cnt[q];
+                            if (n > CAP - 2 * MB) {
+                                const int nn = n < CAP ? n : CAP;
+                                uint64_t *lst = lists + (size_t)q * CAP;
+                                const uint64_t kth = idx::warp_kth_largest(lst, nn, K, hist, lane);
+                                const int m = idx::warp_compact_ge(lst, nn, kth, lane);
+                                if (lane == 0) {
+                                    s_cnt[q] = m;
+                                    // strict from now on: later blocks lose equal-score ties
+                                    s_thr[q] = nextafterf(key_score((uint32_t)(kth >> 32)),
+                                                          INFINITY);
+                                }
+                                __syncwarp();
+                            }
+                        }
+                    }
+                    epi_sync();
+                    if (etid == 0) *overflow = 0;
+#pragma unroll
+                    for (int x = 0; x < QPT; ++x) th[x] = s_thr[q0 + x];
+                    epi_sync();
+                }
+            }
+
+            // ---- finalise: kb - 1 best, ascending by block, own block last
+            const bool aborted = *abort_flag != 0;
+            if (selw) {
+#pragma unroll 1
+                for (int q = e; q < QT; q += SEL_WARPS) {
+                    const int64_t t = g.t0 + q;
+                    if (t >= a.Tq) break;
+                    const int c = s_c[q];
+                    int n = s_cnt[q] < CAP ? s_cnt[q] : CAP;
+                    uint64_t *lst = lists + (size_t)q * CAP;
+                    if (n > SELBUF) {  // rare: cut the list in place first
+                        const uint64_t kth = idx::warp_kth_largest(lst, n, K, hist, lane);
+                        n = idx::warp_compact_ge(lst, n, kth, lane);
+                    }
+                    for (int x = lane; x < n; x += 32) buf[x] = lst[x];
+                    __syncwarp();
+                    int m = n;
+                    if (n > K) {
+                        const uint64_t kth = idx::warp_kth_largest(buf, n, K, hist, lane);
+                        m = idx::warp_compact_ge(buf, n, kth, lane);
+                    }
+                    // re-key as (block << 32 | score key) and sort by block
+                    for (int x = lane; x < m; x += 32) {
+                        const uint64_t k = buf[x];
+                        buf[x] = ((uint64_t)(uint32_t)idx::key_block(k) << 32) | (k >> 32);
+                    }
+                    __syncwarp();
+                    const uint64_t *sorted = idx::warp_radix_sort_hi32(buf, buf + SELBUF / 2, m,
+                                                                       sort_passes, hist, lane);
+                    if (!aborted) {
+                        int32_t *srow = a.sel + ((int64_t)g.b * a.Tq + t) * a.kb;
+                        float *sc = a.sel_score ? a.sel_score + ((int64_t)g.b * a.Tq + t) * a.kb
+                                                : nullptr;
+                        for (int x = lane; x < a.kb; x += 32) {
+                            int32_t id;
+                            float v;
+                            if (x < m) {
+                                id = (int32_t)(sorted[x] >> 32);
+                                v = key_score((uint32_t)sorted[x]);
+                            } else if (x == m) {
+                                id = c;
+                                v = INFINITY;
+                            } else {
+                                id = -1;
+                                v = -INFINITY;
+                            }
+                            srow[x] = id;
+                            if (sc) sc[x] = v;
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+            epi_sync();
+        }
+    }
+
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem_base, 2 * L<HI, DI>::NCOL);
+    }
+}
+
+// ------------------------------------------------------------------- host --
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols innermost, contiguous), box [box_rows, cols].
+static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t cols,
+                     uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw =
+        cols * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static uint32_t wait_limit() {
+    static uint32_t lim = [] {
+        const char *s = getenv("QSA_DEBUG_WAIT_LIMIT");
+        return s ? (uint32_t)strtoul(s, nullptr, 10) : (1u << 22);
+    }();
+    return lim;
+}
+
+template <int HI>
+static int grid_for(int B, int64_t Tq) {
+    const int64_t qt = L<HI, 64>::QT;
+    const int64_t tiles = (int64_t)B * ((Tq + qt - 1) / qt);
+    return (int)(tiles < MAX_GRID ? (tiles > 0 ? tiles : 1) : MAX_GRID);
+}
+
+template <int HI>
+static size_t ws_bytes(int B, int64_t Tq) {
+    const size_t per_cta = (size_t)L<HI, 64>::QT * (CAP * 8 + MAX_GROUPS * MB * 4);
+    return kWsHeader + (size_t)grid_for<HI>(B, Tq) * per_cta;
+}
+
+template <int HI, int DI>
+static cudaError_t launch(const uint16_t *q_idx, const float *w, const uint16_t *kp,
+                          const int64_t *q_pos0, int B, int64_t Tq, int64_t n_blocks, int kb,
+                          int32_t *sel, float *sel_score, void *ws, int num_sms,
+                          cudaStream_t s) {
+    using Lx = L<HI, DI>;
+    auto kern = idx_tc_kernel<HI, DI>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lx::ALLOC);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tm_kp, tm_q;
+    if (!make_map(&tm_kp, kp, (uint64_t)B * (uint64_t)n_blocks, DI, MB) ||
+        !make_map(&tm_q, q_idx, (uint64_t)B * (uint64_t)Tq * HI, DI, Lx::NCOL))
+        return cudaErrorInvalidValue;
+    Args a;
+    a.w = w;
+    a.q_pos0 = q_pos0;
+    a.B = B;
+    a.Tq = Tq;
+    a.n_blocks = n_blocks;
+    a.kb = kb;
+    a.sel = sel;
+    a.sel_score = sel_score;
+    a.ws = static_cast<uint8_t *>(ws);
+    a.n_qt = (int)((Tq + Lx::QT - 1) / Lx::QT);
+    a.total_tiles = a.n_qt * B;
+    a.wait_limit = wait_limit();
+    a.grid = grid_for<HI>(B, Tq);  // the workspace is laid out for this many CTAs
+    int grid = a.grid < num_sms ? a.grid : num_sms;
+    kern<<<grid, THREADS, Lx::ALLOC, s>>>(tm_kp, tm_q, a);
+    return cudaGetLastError();
+}
+
+}  // namespace itc
+
+size_t index_tc_ws_bytes(int B, int64_t Tq, int Hi) {
+    if (Hi == 1) return itc::ws_bytes<1>(B, Tq);
+    if (Hi == 2) return itc::ws_bytes<2>(B, Tq);
+    return itc::ws_bytes<4>(B, Tq);
+}
+
+int index_tc_grid(int B, int64_t Tq, int Hi) {
+    if (Hi == 1) return itc::grid_for<1>(B, Tq);
+    if (Hi == 2) return itc::grid_for<2>(B, Tq);
+    return itc::grid_for<4>(B, Tq);
+}
+
+int index_tc_max_keep() { return itc::MAX_KEEP; }
+
+cudaError_t launch_index_topk_tc(const uint16_t *q_idx, const float *w, const uint16_t *kp,
+                                 const int64_t *q_pos0, int B, int64_t Tq, int64_t n_blocks,
+                                 int Hi, int Di, int kb, int32_t *sel, float *sel_score, void *ws,
+                                 int num_sms, cudaStream_t s) {
+#define QSA_ITC(HI_, DI_)        \
+    if (Hi == HI_ && Di == DI_)  \
+        return itc::launch<HI_, DI_>(q_idx, w, kp, q_pos0, B, Tq, n_blocks, kb, sel, sel_score, \
+                                     ws, num_sms, s);
+    QSA_ITC(1, 32) QSA_ITC(2, 32) QSA_ITC(4, 32) QSA_ITC(1, 64) QSA_ITC(2, 64) QSA_ITC(4, 64)
+#undef QSA_ITC
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace qsa

@@ -15,7 +15,6 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxIndexGrid = 320;  // persistent indexer CTAs (workspace is sized for it)
 constexpr size_t kHeader = 256;
 
 struct DeviceInfo {
@@ -74,12 +73,6 @@ bool supported_indexer(int Hi, int Di) {
 }
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
-
-// Index workspace: header + candidate lists of the persistent CTAs.
-int index_grid_for(int B, int64_t Tq) {
-    const int64_t tiles = (int64_t)B * cdiv(Tq, 64);
-    return (int)(tiles < kMaxIndexGrid ? (tiles > 0 ? tiles : 1) : kMaxIndexGrid);
-}
 
 int sparse_decode_nsplit(int B, int kb) {
     int ns = (int)cdiv(512, B > 0 ? B : 1);
@@ -141,9 +134,8 @@ size_t qsa_index_topk_workspace_size(int B, int64_t Tq, int64_t n_blocks, int Hi
     if (B < 1 || Tq < 0 || n_blocks < 0 || Hi < 1 || Di < 1 || r < 1 || budget < r ||
         budget % r != 0)
         return SIZE_MAX;
-    (void)Hi;
     (void)Di;
-    return qsa::index_topk_ws_bytes(index_grid_for(B, Tq));
+    return qsa::index_tc_ws_bytes(B, Tq, Hi);
 }
 
 qsa_status_t qsa_index_topk(const qsa_bf16_t *q_idx, const float *w, const qsa_bf16_t *k_pooled,
@@ -157,20 +149,17 @@ qsa_status_t qsa_index_topk(const qsa_bf16_t *q_idx, const float *w, const qsa_b
     if (!q_idx || !w || !k_pooled || !sel) return QSA_ERR_INVALID_ARG;
     if (!q_pos0 && (Tq - 1) / r > n_blocks) return QSA_ERR_INVALID_ARG;
     const int kb = budget / r;
-    if (r != 4 || !supported_indexer(Hi, Di) || kb - 1 > qsa::index_topk_max_keep())
+    if (r != 4 || !supported_indexer(Hi, Di) || kb - 1 > qsa::index_tc_max_keep())
         return QSA_ERR_UNSUPPORTED_SHAPE;
-    const int grid = index_grid_for(B, Tq);
-    if (!ws || ws_bytes < qsa::index_topk_ws_bytes(grid) || !aligned16(ws))
+    if (!ws || ws_bytes < qsa::index_tc_ws_bytes(B, Tq, Hi) || !aligned16(ws))
         return QSA_ERR_WORKSPACE;
     if (!aligned16(q_idx) || !aligned16(k_pooled)) return QSA_ERR_INVALID_ARG;
     int sms = 0;
     qsa_status_t st = current_device(&sms);
     if (st != QSA_OK) return st;
-    int g = qsa::index_topk_grid(sms);
-    if (g > grid) g = grid;
-    return from_cuda(qsa::launch_index_topk(q_idx, w, k_pooled, q_pos0, B, Tq, n_blocks, Hi, Di,
-                                            kb, sel, sel_score, ws, g,
-                                            static_cast<cudaStream_t>(stream)));
+    return from_cuda(qsa::launch_index_topk_tc(q_idx, w, k_pooled, q_pos0, B, Tq, n_blocks, Hi,
+                                               Di, kb, sel, sel_score, ws, sms,
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 size_t qsa_index_topk_decode_workspace_size(int B, int64_t n_blocks, int r, int budget) {
@@ -187,7 +176,7 @@ qsa_status_t qsa_index_topk_decode(const qsa_bf16_t *q_idx, const float *w,
         return QSA_ERR_INVALID_ARG;
     if (!q_idx || !w || !k_pooled || !seqlens || !sel) return QSA_ERR_INVALID_ARG;
     const int kb = budget / r;
-    if (r != 4 || !supported_indexer(Hi, Di) || kb - 1 > qsa::index_topk_max_keep() ||
+    if (r != 4 || !supported_indexer(Hi, Di) || kb - 1 > qsa::index_tc_max_keep() ||
         qsa::index_decode_merge_cap(n_blocks, kb) < 0)
         return QSA_ERR_UNSUPPORTED_SHAPE;
     if (!ws || ws_bytes < qsa::index_decode_ws_bytes(B, n_blocks, kb, 0) || !aligned16(ws))

@@ -10,13 +10,13 @@ namespace qsa {
 cudaError_t launch_pool(const uint16_t *k_idx, int B, int64_t T, int Di, int64_t j0,
                         int64_t j1, uint16_t *kp, cudaStream_t s, int num_sms);
 
-size_t index_topk_ws_bytes(int grid);
-int index_topk_grid(int num_sms);
-int index_topk_max_keep();
-cudaError_t launch_index_topk(const uint16_t *q_idx, const float *w, const uint16_t *kp,
-                              const int64_t *q_pos0, int B, int64_t Tq, int64_t n_blocks,
-                              int Hi, int Di, int kb, int32_t *sel, float *sel_score,
-                              void *ws, int grid, cudaStream_t s);
+int index_tc_grid(int B, int64_t Tq, int Hi);
+size_t index_tc_ws_bytes(int B, int64_t Tq, int Hi);
+int index_tc_max_keep();
+cudaError_t launch_index_topk_tc(const uint16_t *q_idx, const float *w, const uint16_t *kp,
+                                 const int64_t *q_pos0, int B, int64_t Tq, int64_t n_blocks,
+                                 int Hi, int Di, int kb, int32_t *sel, float *sel_score, void *ws,
+                                 int num_sms, cudaStream_t s);
 
 size_t index_decode_ws_bytes(int B, int64_t n_blocks, int kb, int num_sms);
 int index_decode_merge_cap(int64_t n_blocks, int kb);  // -1: too many splits

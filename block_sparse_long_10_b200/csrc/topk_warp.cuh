@@ -1,0 +1,213 @@
+// Warp-level exact top-k helpers over unique 64-bit keys (order-preserving
+// score bits above the complemented block index), shared by the indexers.
+#pragma once
+
+#include "qsa_common.cuh"
+
+namespace qsa {
+namespace idx {
+
+// Warp-aggregated histogram increment: lanes with equal digits add once.
+QSA_DEVICE void hist_add(uint32_t *hist, uint32_t digit, bool active, int lane) {
+    const uint32_t act = __ballot_sync(0xffffffffu, active);
+    if (!active) return;
+    const uint32_t peers = __match_any_sync(act, digit);
+    if (__ffs(peers) - 1 == lane) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+}
+
+QSA_DEVICE uint64_t warp_min_u64(uint64_t v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+        v = o < v ? o : v;
+    }
+    return v;
+}
+QSA_DEVICE uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+        v = o > v ? o : v;
+    }
+    return v;
+}
+
+// Radix select: the K-th largest of n unique keys (1 <= K <= n) in `buf`
+// (shared or global memory).  The first 8-bit digit sits just below the
+// highest bit on which the keys differ; later digits follow; the search stops
+// as soon as the bucket holding the K-th key is kept whole (its minimum is
+// then the answer).
+QSA_DEVICE uint64_t warp_kth_largest(const uint64_t *buf, int n, int K, uint32_t *hist,
+                                     int lane) {
+    uint64_t mn = ~0ull, mx = 0ull;
+    for (int i = lane; i < n; i += 32) {
+        const uint64_t k = buf[i];
+        mn = k < mn ? k : mn;
+        mx = k > mx ? k : mx;
+    }
+    mn = warp_min_u64(mn);
+    mx = warp_max_u64(mx);
+    if (mn == mx || K >= n) return mn;
+    if (K == 1) return mx;
+    int top = 63 - __clzll((long long)(mn ^ mx));      // highest differing bit
+    uint64_t prefix = top >= 63 ? 0ull : (mn & (~0ull << (top + 1)));
+    int want = K;
+#pragma unroll 1
+    for (;;) {
+        const int shift = top - 7;                       // window [shift, top]
+        const uint64_t hm = top >= 63 ? 0ull : (~0ull << (top + 1));
+        for (int i = lane; i < 256; i += 32) hist[i] = 0;
+        __syncwarp();
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            const uint64_t k = i < n ? buf[i] : 0ull;
+            const bool m = i < n && (k & hm) == prefix;
+            const uint32_t d = (uint32_t)((shift >= 0 ? (k >> shift) : (k << -shift)) & 255u);
+            hist_add(hist, d, m, lane);
+        }
+        __syncwarp();
+        uint32_t local[8];
+        uint32_t sum = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            local[b] = hist[lane * 8 + b];
+            sum += local[b];
+        }
+        uint32_t incl = sum;  // keys in this lane's bins and above
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+            if (lane + off < 32) incl += y;
+        }
+        uint32_t cum = incl - sum;
+        int found = -1, new_want = 0;
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int b = 7; b >= 0; --b) {
+            if (found < 0 && (int)cum < want && want <= (int)(cum + local[b])) {
+                found = lane * 8 + b;
+                new_want = want - (int)cum;
+                cnt = local[b];
+            }
+            cum += local[b];
+        }
+        const uint32_t ball = __ballot_sync(0xffffffffu, found >= 0);
+        const int src = __ffs(ball) - 1;
+        found = __shfl_sync(0xffffffffu, found, src);
+        want = __shfl_sync(0xffffffffu, new_want, src);
+        cnt = __shfl_sync(0xffffffffu, cnt, src);
+        prefix |= shift >= 0 ? ((uint64_t)(uint32_t)found << shift)
+                             : ((uint64_t)(uint32_t)found >> -shift);
+        __syncwarp();
+        if (shift <= 0) return prefix;                   // every bit decided
+        if ((int)cnt == want) {                          // bucket kept whole
+            const uint64_t m2 = ~0ull << shift;
+            uint64_t bmin = ~0ull;
+            for (int i = lane; i < n; i += 32) {
+                const uint64_t k = buf[i];
+                if ((k & m2) == prefix && k < bmin) bmin = k;
+            }
+            return warp_min_u64(bmin);
+        }
+        top = shift - 1;
+    }
+}
+
+// Keep the keys >= kth (exactly K of them) at the front of buf; returns count.
+QSA_DEVICE int warp_compact_ge(uint64_t *buf, int n, uint64_t kth, int lane) {
+    int base = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const uint64_t k = (i < n) ? buf[i] : 0ull;
+        const bool keep = (i < n) && (k >= kth);
+        const uint32_t m = __ballot_sync(0xffffffffu, keep);
+        if (keep) buf[base + __popc(m & ((1u << lane) - 1u))] = k;
+        base += __popc(m);
+    }
+    __syncwarp();
+    return base;
+}
+
+// Stable copy of the keys >= kth from src to dst; returns how many.
+QSA_DEVICE int warp_copy_ge(uint64_t *dst, const uint64_t *src, int n, uint64_t kth, int lane) {
+    int base = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const uint64_t k = (i < n) ? src[i] : 0ull;
+        const bool keep = (i < n) && (k >= kth);
+        const uint32_t m = __ballot_sync(0xffffffffu, keep);
+        if (keep) dst[base + __popc(m & ((1u << lane) - 1u))] = k;
+        base += __popc(m);
+    }
+    __syncwarp();
+    return base;
+}
+
+// Stable LSD radix sort (8-bit digits) of m <= 1024 keys by their high 32
+// bits, which hold values below 2^(8*passes).  Ping-pongs between buf and
+// tmp; returns the buffer that holds the result.
+QSA_DEVICE uint64_t *warp_radix_sort_hi32(uint64_t *buf, uint64_t *tmp, int m, int passes,
+                                          uint32_t *hist, int lane) {
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 1
+    for (int p = 0; p < passes; ++p) {
+        const int sh = 32 + 8 * p;
+        for (int i = lane; i < 256; i += 32) hist[i] = 0;
+        __syncwarp();
+        for (int i0 = 0; i0 < m; i0 += 32) {
+            const int i = i0 + lane;
+            const uint64_t k = i < m ? buf[i] : 0ull;
+            hist_add(hist, (uint32_t)(k >> sh) & 255u, i < m, lane);
+        }
+        __syncwarp();
+        // exclusive prefix sum over the 256 bins
+        uint32_t local[8], sum = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            local[b] = hist[lane * 8 + b];
+            sum += local[b];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        uint32_t run = incl - sum;
+        __syncwarp();
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            hist[lane * 8 + b] = run;
+            run += local[b];
+        }
+        __syncwarp();
+        for (int i0 = 0; i0 < m; i0 += 32) {
+            const int i = i0 + lane;
+            const bool v = i < m;
+            const uint64_t k = v ? buf[i] : 0ull;
+            const uint32_t d = (uint32_t)(k >> sh) & 255u;
+            const uint32_t act = __ballot_sync(0xffffffffu, v);
+            uint32_t peers = 0, base = 0;
+            if (v) {
+                peers = __match_any_sync(act, d);
+                base = hist[d];
+                tmp[base + __popc(peers & lt)] = k;
+            }
+            __syncwarp();
+            if (v && __ffs(peers) - 1 == lane) hist[d] = base + __popc(peers);
+            __syncwarp();
+        }
+        uint64_t *x = buf;
+        buf = tmp;
+        tmp = x;
+    }
+    return buf;
+}
+
+QSA_DEVICE uint64_t make_key(float s, int j) {
+    return ((uint64_t)score_key(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+}
+QSA_DEVICE int key_block(uint64_t k) { return (int)(0xFFFFFFFFu - (uint32_t)k); }
+
+}  // namespace idx
+}  // namespace qsa
