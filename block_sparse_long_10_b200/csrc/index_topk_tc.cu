@@ -55,6 +55,7 @@ constexpr int SEL_WARPS = 8;     // epilogue warps that also run the selections
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr int CAP = 2048;        // candidate-list capacity per query (workspace)
 constexpr int SELBUF = 1024;     // per selecting warp, u64 keys in shared memory
+constexpr int CHECK_EVERY = 8;   // pass-2 tiles between list-capacity checks
 constexpr int MAX_GROUPS = 8;    // group maxima per block lane and query
 constexpr int MAX_KEEP = 511;
 constexpr int MAX_GRID = 160;
@@ -92,7 +93,7 @@ struct Args {
     float *sel_score;
     uint8_t *ws;
     int n_qt, total_tiles;
-    uint32_t wait_limit;
+    uint64_t wait_limit;  // ns
     int grid;
 };
 
@@ -232,12 +233,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // let this CTA's own copies in flight land before it exits (bounded)
                 for (int s2 = 0; s2 < STAGES; ++s2)
                     if (last_kp[s2] >= 0)
-                        for (uint32_t n = 0; n < (1u << 20); ++n)
-                            if (sm100::mbar_try_wait(&full[s2], (last_kp[s2] / STAGES) & 1)) break;
+                        sm100::mbar_wait_for(&full[s2], (last_kp[s2] / STAGES) & 1, 100000000ull);
                 for (int qb = 0; qb < 2; ++qb)
                     if (last_q[qb] >= 0)
-                        for (uint32_t n = 0; n < (1u << 20); ++n)
-                            if (sm100::mbar_try_wait(&qfull[qb], (last_q[qb] >> 1) & 1)) break;
+                        sm100::mbar_wait_for(&qfull[qb], (last_q[qb] >> 1) & 1, 100000000ull);
             }
         }
     } else if (warp == 1) {
@@ -278,8 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             // every MMA this thread issued has retired before TMEM is freed (bounded)
             sm100::mma_commit(mma_done);
-            for (uint32_t n = 0; n < (1u << 22); ++n)
-                if (sm100::mbar_try_wait(mma_done, 0)) break;
+            sm100::mbar_wait_for(mma_done, 0, 1000000000ull);
         }
     } else {
         // ------------------------------------------------------ epilogue --
@@ -329,16 +327,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const bool tail = (int64_t)kt * MB + MB > g.c_min;
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
+                {
+                    constexpr int NCH = NCOL / 4 / 32;  // 32-column chunks per thread (1 or 2)
+                    uint32_t v[NCH][32];
+                    if constexpr (NCH == 2)
+                        sm100::tmem_ld32x2(taddr, taddr + 32, v[0], v[NCH - 1]);
+                    else
+                        sm100::tmem_ld32(taddr, v[0]);
 #pragma unroll
-                for (int ch = 0; ch < NCOL / 4 / 32; ++ch) {
-                    uint32_t v[32];
-                    sm100::tmem_ld32(taddr + ch * 32, v);
+                    for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
-                    for (int qq = 0; qq < 32 / HI; ++qq) {
-                        const int x = ch * (32 / HI) + qq;
-                        const float s = score_of<HI>(v + qq * HI, s_w[q0 + x]);
-                        if (!tail || j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], s);
-                    }
+                        for (int qq = 0; qq < 32 / HI; ++qq) {
+                            const int x = ch * (32 / HI) + qq;
+                            const float s = score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]);
+                            if (!tail || j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], s);
+                        }
                 }
                 sm100::tc_fence_before();
                 __syncwarp();
@@ -387,32 +390,40 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const bool tail = (int64_t)kt * MB + MB > g.c_min;
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
+                {
+                    constexpr int NCH = NCOL / 4 / 32;  // 32-column chunks per thread (1 or 2)
+                    uint32_t v[NCH][32];
+                    if constexpr (NCH == 2)
+                        sm100::tmem_ld32x2(taddr, taddr + 32, v[0], v[NCH - 1]);
+                    else
+                        sm100::tmem_ld32(taddr, v[0]);
 #pragma unroll
-                for (int ch = 0; ch < NCOL / 4 / 32; ++ch) {
-                    uint32_t v[32];
-                    sm100::tmem_ld32(taddr + ch * 32, v);
+                    for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
-                    for (int qq = 0; qq < 32 / HI; ++qq) {
-                        const int x = ch * (32 / HI) + qq;
-                        const float s = score_of<HI>(v + qq * HI, s_w[q0 + x]);
-                        if (s >= th[x] && (!tail || j < s_c[q0 + x])) {
-                            const int pos = atomicAdd(&s_cnt[q0 + x], 1);
-                            if (pos < CAP)
-                                lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(s, j);
-                            if (pos == CAP - 2 * MB) *overflow = 1;
+                        for (int qq = 0; qq < 32 / HI; ++qq) {
+                            const int x = ch * (32 / HI) + qq;
+                            const float s = score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]);
+                            if (s >= th[x] && (!tail || j < s_c[q0 + x])) {
+                                const int pos = atomicAdd(&s_cnt[q0 + x], 1);
+                                if (pos < CAP)
+                                    lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(s, j);
+                                if (pos == CAP - CHECK_EVERY * MB) *overflow = 1;
+                            }
                         }
-                    }
                 }
                 sm100::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) sm100::mbar_arrive(&tempty[tb]);
+                // lists are checked every CHECK_EVERY tiles: a list below
+                // CAP - CHECK_EVERY * MB at a check cannot overflow before the next
+                if ((kt + 1) % CHECK_EVERY != 0 && kt + 1 != g.n_kt) continue;
                 epi_sync();
                 if (*overflow) {  // uniform: read after the barrier, set only before it
                     if (selw) {
 #pragma unroll 1
                         for (int q = e; q < QT; q += SEL_WARPS) {
                             const int n = s_cnt[q];
-                            if (n > CAP - 2 * MB) {
+                            if (n > CAP - CHECK_EVERY * MB) {
                                 const int nn = n < CAP ? n : CAP;
                                 uint64_t *lst = lists + (size_t)q * CAP;
                                 const uint64_t kth = idx::warp_kth_largest(lst, nn, K, hist, lane);
@@ -538,10 +549,12 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t c
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static uint32_t wait_limit() {
-    static uint32_t lim = [] {
-        const char *s = getenv("QSA_DEBUG_WAIT_LIMIT");
-        return s ? (uint32_t)strtoul(s, nullptr, 10) : (1u << 22);
+// Bound on any single wait inside the kernel (ns); QSA_DEBUG_WAIT_NS overrides
+// it so tests can make a wait run out on purpose.
+static uint64_t wait_limit() {
+    static uint64_t lim = [] {
+        const char *s = getenv("QSA_DEBUG_WAIT_NS");
+        return s ? (uint64_t)strtoull(s, nullptr, 10) : 2000000000ull;
     }();
     return lim;
 }
