@@ -370,7 +370,20 @@ def extra_prefill(qsa, name, device, peaks, flush):
     dense = time_call(lambda: qsa.qsa_dense_gqa_prefill(x["q"], x["k"], x["v"], o, w.scale),
                       run.stream, 2, 1, flush)
     rep, wk = kernel_report(w, kern, peaks)
+    sdpa = None
+    try:  # torch's own fused attention (flash / cuDNN) on the same tensors, for context
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        qt = x["q"].transpose(1, 2)
+        kt = x["k"].repeat_interleave(w.G, dim=2).transpose(1, 2)
+        vt = x["v"].repeat_interleave(w.G, dim=2).transpose(1, 2)
+        with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.CUDNN_ATTENTION]):
+            sdpa = time_call(lambda: torch.nn.functional.scaled_dot_product_attention(
+                qt, kt, vt, is_causal=True, scale=w.scale), run.stream, 2, 1, flush)
+        del qt, kt, vt
+    except Exception as exc:  # no fused backend for this shape: report why
+        sdpa = f"unavailable: {type(exc).__name__}"
     out = {"ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3), "kernels": rep,
+           "torch_sdpa_dense_ms": sdpa,
            "dense_gqa_ms": dense,
            "dense_gqa_tflops": wk["dense_flops"] / (dense / 1e3) / 1e12,
            "dense_frac_tensor": wk["dense_flops"] / (dense / 1e3) / 1e12 / peaks["bf16_tflops"],

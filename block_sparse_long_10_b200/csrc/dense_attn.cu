@@ -219,8 +219,7 @@ static cudaError_t launch_dense(const uint16_t *q, const uint16_t *k, const uint
                                 cudaStream_t s) {
     using C = Cfg<D>;
     auto kern = dense_prefill_kernel<D, G>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
     if (e != cudaSuccess) return e;
     constexpr int TOK = ROWS / G;
     const int n_qt = (int)((T + TOK - 1) / TOK);

@@ -38,8 +38,6 @@
 // because blocks are swept in ascending order.  Scores never reach HBM.
 #include <stdlib.h>
 
-#include <mutex>
-
 #include "qsa_common.cuh"
 #include "qsa_launch.h"
 #include "sm100.cuh"
@@ -512,43 +510,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ------------------------------------------------------------------- host --
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        else
-            cudaGetLastError();
-    });
-    return fn;
-}
-
-// 2-D bf16 tensor [rows, cols] (cols innermost, contiguous), box [box_rows, cols].
-static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t cols,
-                     uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {cols, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapSwizzle sw =
-        cols * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Bound on any single wait inside the kernel (ns); QSA_DEBUG_WAIT_NS overrides
 // it so tests can make a wait run out on purpose.
 static uint64_t wait_limit() {
@@ -579,12 +540,11 @@ static cudaError_t launch(const uint16_t *q_idx, const float *w, const uint16_t 
                           cudaStream_t s) {
     using Lx = L<HI, DI>;
     auto kern = idx_tc_kernel<HI, DI>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lx::ALLOC);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), Lx::ALLOC);
     if (e != cudaSuccess) return e;
     CUtensorMap tm_kp, tm_q;
-    if (!make_map(&tm_kp, kp, (uint64_t)B * (uint64_t)n_blocks, DI, MB) ||
-        !make_map(&tm_q, q_idx, (uint64_t)B * (uint64_t)Tq * HI, DI, Lx::NCOL))
+    if (!tensor_map_2d_bf16(&tm_kp, kp, (uint64_t)B * (uint64_t)n_blocks, DI, MB) ||
+        !tensor_map_2d_bf16(&tm_q, q_idx, (uint64_t)B * (uint64_t)Tq * HI, DI, Lx::NCOL))
         return cudaErrorInvalidValue;
     Args a;
     a.w = w;

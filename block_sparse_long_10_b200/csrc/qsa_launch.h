@@ -5,7 +5,14 @@
 #include <stddef.h>
 #include <stdint.h>
 
+struct CUtensorMap_st;
+
 namespace qsa {
+
+// Host caches (host_util.cu).
+cudaError_t ensure_smem(const void *kern, int bytes);
+bool tensor_map_2d_bf16(CUtensorMap_st *out, const void *base, uint64_t rows, uint32_t cols,
+                        uint32_t box_rows);
 
 cudaError_t launch_pool(const uint16_t *k_idx, int B, int64_t T, int Di, int64_t j0,
                         int64_t j1, uint16_t *kp, cudaStream_t s, int num_sms);

@@ -323,8 +323,7 @@ template <int D, int G, int HKV, int MODE>
 static cudaError_t launch_sat(const Args &a, int grid, cudaStream_t s) {
     using C = Cfg<D, HKV>;
     auto kern = sparse_attn_kernel<D, G, HKV, MODE>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
     if (e != cudaSuccess) return e;
     if (a.total_items == 0) return cudaSuccess;
     kern<<<grid, THREADS, C::BYTES, s>>>(a);

@@ -7,12 +7,12 @@
 namespace qsa {
 namespace idx {
 
-// Warp-aggregated histogram increment: lanes with equal digits add once.
+// Histogram increment.  The radix passes start at the highest bit on which
+// the keys differ, so digits spread over the bins and plain shared atomics
+// see little contention.
 QSA_DEVICE void hist_add(uint32_t *hist, uint32_t digit, bool active, int lane) {
-    const uint32_t act = __ballot_sync(0xffffffffu, active);
-    if (!active) return;
-    const uint32_t peers = __match_any_sync(act, digit);
-    if (__ffs(peers) - 1 == lane) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+    (void)lane;
+    if (active) atomicAdd(&hist[digit], 1u);
 }
 
 QSA_DEVICE uint64_t warp_min_u64(uint64_t v) {
