@@ -70,6 +70,7 @@ struct L {
     static constexpr int OFF_Q = OFF_KP + STAGES * KP_TILE;
     static constexpr int OFF_BUF = OFF_Q + 2 * Q_TILE;
     static constexpr int OFF_HIST = OFF_BUF + SEL_WARPS * SELBUF * 8;
+    static_assert(EPI_WARPS * QPT * 32 * 4 <= SEL_WARPS * SELBUF * 8, "pass-2 score park");
     static constexpr int OFF_W = OFF_HIST + SEL_WARPS * 256 * 4;
     static constexpr int OFF_THR = OFF_W + QT * 16;
     static constexpr int OFF_C = OFF_THR + QT * 4;
@@ -130,13 +131,38 @@ QSA_DEVICE TileGeo tile_geo(const Args &a, int tile) {
     return g;
 }
 
+QSA_DEVICE uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+QSA_DEVICE float f2_sum(uint64_t p) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+    return lo + hi;
+}
+
+// s = sum_h w_h * max(x_h, 0) in fp32, heads paired on the packed f32x2 pipe:
+// (w0 r0 + w2 r2) + (w1 r1 + w3 r3).  Both passes call this same function, so
+// a block's score is bit-identical in them.
 template <int HI>
 QSA_DEVICE float score_of(const uint32_t *v, const float4 wq) {
-    const float wa[4] = {wq.x, wq.y, wq.z, wq.w};
-    float s = 0.f;
-#pragma unroll
-    for (int h = 0; h < HI; ++h) s = fmaf(wa[h], fmaxf(__uint_as_float(v[h]), 0.f), s);
-    return s;
+    const float r0 = fmaxf(__uint_as_float(v[0]), 0.f);
+    if constexpr (HI == 1) {
+        return wq.x * r0;
+    } else {
+        const float r1 = fmaxf(__uint_as_float(v[1]), 0.f);
+        uint64_t acc;
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(acc) : "l"(f2_pack(wq.x, wq.y)), "l"(f2_pack(r0, r1)));
+        if constexpr (HI == 4) {
+            const float r2 = fmaxf(__uint_as_float(v[2]), 0.f);
+            const float r3 = fmaxf(__uint_as_float(v[3]), 0.f);
+            asm("fma.rn.f32x2 %0, %1, %2, %0;"
+                : "+l"(acc)
+                : "l"(f2_pack(wq.z, wq.w)), "l"(f2_pack(r2, r3)));
+        }
+        return f2_sum(acc);
+    }
 }
 
 template <int HI, int DI>
@@ -332,14 +358,24 @@ __global__ void __launch_bounds__(THREADS, 1)
                         sm100::tmem_ld32x2(taddr, taddr + 32, v[0], v[NCH - 1]);
                     else
                         sm100::tmem_ld32(taddr, v[0]);
+                    if (!tail) {
 #pragma unroll
-                    for (int ch = 0; ch < NCH; ++ch)
+                        for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
-                        for (int qq = 0; qq < 32 / HI; ++qq) {
-                            const int x = ch * (32 / HI) + qq;
-                            const float s = score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]);
-                            if (!tail || j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], s);
-                        }
+                            for (int qq = 0; qq < 32 / HI; ++qq) {
+                                const int x = ch * (32 / HI) + qq;
+                                gm[x] = fmaxf(gm[x], score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]));
+                            }
+                    } else {
+#pragma unroll
+                        for (int ch = 0; ch < NCH; ++ch)
+#pragma unroll
+                            for (int qq = 0; qq < 32 / HI; ++qq) {
+                                const int x = ch * (32 / HI) + qq;
+                                const float s = score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]);
+                                if (j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], s);
+                            }
+                    }
                 }
                 sm100::tc_fence_before();
                 __syncwarp();
@@ -377,9 +413,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             epi_sync();
 
             // ---- pass 2: keep every candidate with s >= theta ------------
-            float th[QPT];
+            // s >= theta  <=>  s > below(theta), read off the sign of
+            // below(theta) - s (exact: the difference of two floats is zero only
+            // when they are equal)
+            float thp[QPT];
 #pragma unroll
-            for (int x = 0; x < QPT; ++x) th[x] = s_thr[q0 + x];
+            for (int x = 0; x < QPT; ++x) thp[x] = nextafterf(s_thr[q0 + x], -INFINITY);
+            // this warp's survivor scores, [query x][lane]: the selection buffers
+            // are idle during pass 2 (16 warps x QPT x 32 floats fit in them)
+            float *scw = reinterpret_cast<float *>(sm + Lx::OFF_BUF) + e * (QPT * 32);
             for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
                 const int tb = it & 1;
                 sm100::mbar_wait(&tfull[tb], (it >> 1) & 1, abort_flag, a.wait_limit, a.ws);
@@ -395,19 +437,30 @@ __global__ void __launch_bounds__(THREADS, 1)
                         sm100::tmem_ld32x2(taddr, taddr + 32, v[0], v[NCH - 1]);
                     else
                         sm100::tmem_ld32(taddr, v[0]);
+                    // bit QPT-1-x of hit: query x keeps this block; the score of a
+                    // survivor is parked in shared memory (predicated store, no
+                    // branch per pair)
+                    uint32_t hit = 0;
 #pragma unroll
                     for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
                         for (int qq = 0; qq < 32 / HI; ++qq) {
                             const int x = ch * (32 / HI) + qq;
                             const float s = score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]);
-                            if (s >= th[x] && (!tail || j < s_c[q0 + x])) {
-                                const int pos = atomicAdd(&s_cnt[q0 + x], 1);
-                                if (pos < CAP)
-                                    lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(s, j);
-                                if (pos == CAP - CHECK_EVERY * MB) *overflow = 1;
-                            }
+                            const bool keep = s > thp[x];
+                            hit = (hit << 1) | (uint32_t)keep;
+                            if (keep) scw[x * 32 + lane] = s;
                         }
+                    while (hit) {  // rare: about one survivor per 20 (thread, tile)
+                        const int b = 31 - __clz(hit);
+                        hit &= ~(1u << b);
+                        const int x = QPT - 1 - b;
+                        if (tail && j >= s_c[q0 + x]) continue;
+                        const int pos = atomicAdd(&s_cnt[q0 + x], 1);
+                        if (pos < CAP)
+                            lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(scw[x * 32 + lane], j);
+                        if (pos == CAP - CHECK_EVERY * MB) *overflow = 1;
+                    }
                 }
                 sm100::tc_fence_before();
                 __syncwarp();
@@ -439,7 +492,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     epi_sync();
                     if (etid == 0) *overflow = 0;
 #pragma unroll
-                    for (int x = 0; x < QPT; ++x) th[x] = s_thr[q0 + x];
+                    for (int x = 0; x < QPT; ++x) thp[x] = nextafterf(s_thr[q0 + x], -INFINITY);
                     epi_sync();
                 }
             }
