@@ -413,9 +413,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             epi_sync();
 
             // ---- pass 2: keep every candidate with s >= theta ------------
-            // s >= theta  <=>  s > below(theta), read off the sign of
-            // below(theta) - s (exact: the difference of two floats is zero only
-            // when they are equal)
+            // s >= theta  <=>  s > below(theta), the next float down
             float thp[QPT];
 #pragma unroll
             for (int x = 0; x < QPT; ++x) thp[x] = nextafterf(s_thr[q0 + x], -INFINITY);
@@ -430,6 +428,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const bool tail = (int64_t)kt * MB + MB > g.c_min;
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
+                uint32_t hit = 0;
                 {
                     constexpr int NCH = NCOL / 4 / 32;  // 32-column chunks per thread (1 or 2)
                     uint32_t v[NCH][32];
@@ -440,7 +439,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     // bit QPT-1-x of hit: query x keeps this block; the score of a
                     // survivor is parked in shared memory (predicated store, no
                     // branch per pair)
-                    uint32_t hit = 0;
 #pragma unroll
                     for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
@@ -451,20 +449,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                             hit = (hit << 1) | (uint32_t)keep;
                             if (keep) scw[x * 32 + lane] = s;
                         }
-                    while (hit) {  // rare: about one survivor per 20 (thread, tile)
-                        const int b = 31 - __clz(hit);
-                        hit &= ~(1u << b);
-                        const int x = QPT - 1 - b;
-                        if (tail && j >= s_c[q0 + x]) continue;
-                        const int pos = atomicAdd(&s_cnt[q0 + x], 1);
-                        if (pos < CAP)
-                            lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(scw[x * 32 + lane], j);
-                        if (pos == CAP - CHECK_EVERY * MB) *overflow = 1;
-                    }
                 }
+                // the TMEM buffer is free before the appends: they only need the
+                // mask and the parked scores
                 sm100::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) sm100::mbar_arrive(&tempty[tb]);
+                while (hit) {  // rare: about one survivor per 20 (thread, tile)
+                    const int b = 31 - __clz(hit);
+                    hit &= ~(1u << b);
+                    const int x = QPT - 1 - b;
+                    if (tail && j >= s_c[q0 + x]) continue;
+                    const int pos = atomicAdd(&s_cnt[q0 + x], 1);
+                    if (pos < CAP)
+                        lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(scw[x * 32 + lane], j);
+                    if (pos == CAP - CHECK_EVERY * MB) *overflow = 1;
+                }
                 // lists are checked every CHECK_EVERY tiles: a list below
                 // CAP - CHECK_EVERY * MB at a check cannot overflow before the next
                 if ((kt + 1) % CHECK_EVERY != 0 && kt + 1 != g.n_kt) continue;
