@@ -43,6 +43,7 @@
 #include "sm100.cuh"
 #include "topk_warp.cuh"
 
+
 namespace qsa {
 namespace itc {
 
@@ -343,6 +344,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             float gm[QPT];
 #pragma unroll
             for (int x = 0; x < QPT; ++x) gm[x] = -INFINITY;
+            int r_in = 0, grp = 0;  // tiles into the current group, group index
             for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
                 const int tb = it & 1;
                 sm100::mbar_wait(&tfull[tb], (it >> 1) & 1, abort_flag, a.wait_limit, a.ws);
@@ -352,41 +354,39 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
                 {
-                    constexpr int NCH = NCOL / 4 / 32;  // 32-column chunks per thread (1 or 2)
-                    uint32_t v[NCH][32];
-                    if constexpr (NCH == 2)
-                        sm100::tmem_ld32x2(taddr, taddr + 32, v[0], v[NCH - 1]);
-                    else
-                        sm100::tmem_ld32(taddr, v[0]);
-                    if (!tail) {
+                    constexpr int CW = 16;  // columns per load: 16 values live at a time
+                    constexpr int NCH = NCOL / 4 / CW;
 #pragma unroll
-                        for (int ch = 0; ch < NCH; ++ch)
+                    for (int ch = 0; ch < NCH; ++ch) {
+                        uint32_t v[CW];
+                        sm100::tmem_ld16(taddr + CW * ch, v);
+                        if (!tail) {
 #pragma unroll
-                            for (int qq = 0; qq < 32 / HI; ++qq) {
-                                const int x = ch * (32 / HI) + qq;
-                                gm[x] = fmaxf(gm[x], score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]));
+                            for (int qq = 0; qq < CW / HI; ++qq) {
+                                const int x = ch * (CW / HI) + qq;
+                                gm[x] = fmaxf(gm[x], score_of<HI>(v + qq * HI, s_w[q0 + x]));
                             }
-                    } else {
+                        } else {
 #pragma unroll
-                        for (int ch = 0; ch < NCH; ++ch)
-#pragma unroll
-                            for (int qq = 0; qq < 32 / HI; ++qq) {
-                                const int x = ch * (32 / HI) + qq;
-                                const float s = score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]);
+                            for (int qq = 0; qq < CW / HI; ++qq) {
+                                const int x = ch * (CW / HI) + qq;
+                                const float s = score_of<HI>(v + qq * HI, s_w[q0 + x]);
                                 if (j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], s);
                             }
+                        }
                     }
                 }
                 sm100::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) sm100::mbar_arrive(&tempty[tb]);
-                if ((kt + 1) % g.R == 0 || kt + 1 == g.n_kt) {
-                    const int grp = kt / g.R;
+                if (++r_in == g.R || kt + 1 == g.n_kt) {
 #pragma unroll
                     for (int x = 0; x < QPT; ++x) {
                         gmax_g[(size_t)(q0 + x) * (MAX_GROUPS * MB) + grp * MB + p] = score_key(gm[x]);
                         gm[x] = -INFINITY;
                     }
+                    r_in = 0;
+                    ++grp;
                 }
             }
             epi_sync();
@@ -430,25 +430,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
                 uint32_t hit = 0;
                 {
-                    constexpr int NCH = NCOL / 4 / 32;  // 32-column chunks per thread (1 or 2)
-                    uint32_t v[NCH][32];
-                    if constexpr (NCH == 2)
-                        sm100::tmem_ld32x2(taddr, taddr + 32, v[0], v[NCH - 1]);
-                    else
-                        sm100::tmem_ld32(taddr, v[0]);
-                    // bit QPT-1-x of hit: query x keeps this block; the score of a
-                    // survivor is parked in shared memory (predicated store, no
-                    // branch per pair)
+                    constexpr int CW = 16;  // columns per load: 16 values live at a time
+                    constexpr int NCH = NCOL / 4 / CW;
 #pragma unroll
-                    for (int ch = 0; ch < NCH; ++ch)
+                    for (int ch = 0; ch < NCH; ++ch) {
+                        uint32_t v[CW];
+                        sm100::tmem_ld16(taddr + CW * ch, v);
 #pragma unroll
-                        for (int qq = 0; qq < 32 / HI; ++qq) {
-                            const int x = ch * (32 / HI) + qq;
-                            const float s = score_of<HI>(v[ch] + qq * HI, s_w[q0 + x]);
+                        for (int qq = 0; qq < CW / HI; ++qq) {
+                            const int x = ch * (CW / HI) + qq;
+                            const float s = score_of<HI>(v + qq * HI, s_w[q0 + x]);
                             const bool keep = s > thp[x];
                             hit = (hit << 1) | (uint32_t)keep;
                             if (keep) scw[x * 32 + lane] = s;
                         }
+                    }
                 }
                 // the TMEM buffer is free before the appends: they only need the
                 // mask and the parked scores
