@@ -10,10 +10,10 @@
 // Work item = one query token (prefill) or one slice of one decode query's
 // selection.  The item's blocks are gathered 4 tokens x all KV heads at a time
 // (one contiguous 2 KiB run per block for K and for V at Hkv = 2, D = 128)
-// with 16-byte cp.async into a 3-stage shared-memory ring, XOR-swizzled for
-// conflict-free ldmatrix.  With G = Hq / Hkv query heads per KV head, a
-// token's work per KV head is M = G rows, too few for an MMA tile, so the MMA
-// runs transposed: S^T = K_sel (16 keys) x Q^T (G <= 8 heads as N = 8).  The
+// with 16-byte cp.async into a shared-memory ring (2 stages in prefill, 3 in
+// decode), XOR-swizzled for conflict-free ldmatrix.  With G = Hq / Hkv query
+// heads per KV head, a token's work per KV head is M = G rows, too few for an
+// MMA tile, so the MMA runs transposed: S^T = K_sel (16 keys) x Q^T (G <= 8 heads as N = 8).  The
 // softmax runs per head column in registers (fp32, base-2 exponent), the
 // probabilities are rounded to bf16 and moved into B-operand layout with
 // movmatrix, and O^T = V_sel^T x P accumulates in fp32.  Warps of one KV head
@@ -29,13 +29,21 @@ namespace sat {
 
 constexpr int WARPS = 4;
 constexpr int THREADS = WARPS * 32;
-constexpr int STAGES = 3;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
 enum Mode { PREFILL = 0, SPLIT = 1 };
 
-template <int D, int HKV>
+// Prefill: 2-stage ring, 3 CTAs per SM (12 warps: the gather is latency-bound
+// and more resident warps beat a deeper ring).  Split decode: 3-stage ring,
+// 2 CTAs per SM (few items per SM, a deeper ring per item pays).
+template <int MODE>
+struct Ring {
+    static constexpr int STAGES = MODE == PREFILL ? 2 : 3;
+    static constexpr int CTAS = MODE == PREFILL ? 3 : 2;
+};
+
+template <int D, int HKV, int STAGES>
 struct Cfg {
     static constexpr int WPG = WARPS / HKV;           // warps per KV head
     static constexpr int KS = 16 * WPG;               // keys per stage
@@ -73,8 +81,9 @@ struct Args {
 };
 
 template <int D, int G, int HKV, int MODE>
-__global__ void __launch_bounds__(THREADS, 2) sparse_attn_kernel(const Args a) {
-    using C = Cfg<D, HKV>;
+__global__ void __launch_bounds__(THREADS, Ring<MODE>::CTAS) sparse_attn_kernel(const Args a) {
+    constexpr int STAGES = Ring<MODE>::STAGES;
+    using C = Cfg<D, HKV, STAGES>;
     constexpr int KSTEP = D / 16;
     extern __shared__ __align__(128) uint8_t smem[];
     int *s_blk = reinterpret_cast<int *>(smem + C::OFF_SEL);
@@ -321,7 +330,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const float *__restr
 
 template <int D, int G, int HKV, int MODE>
 static cudaError_t launch_sat(const Args &a, int grid, cudaStream_t s) {
-    using C = Cfg<D, HKV>;
+    using C = Cfg<D, HKV, Ring<MODE>::STAGES>;
     auto kern = sparse_attn_kernel<D, G, HKV, MODE>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
     if (e != cudaSuccess) return e;
@@ -356,7 +365,7 @@ cudaError_t launch_sparse_attn_prefill(const uint16_t *q, const uint16_t *k, con
     a.B = B; a.Tq = Tq; a.Tk = Tk; a.Hq = Hq; a.kb = kb; a.nsplit = 1; a.chunk = kb;
     a.scale_log2 = scale * sat::LOG2E; a.o = o; a.lse = lse; a.part = nullptr;
     a.status = nullptr; a.total_items = (int64_t)B * Tq;
-    int64_t grid = (int64_t)num_sms * 2;
+    int64_t grid = (int64_t)num_sms * sat::Ring<sat::PREFILL>::CTAS;
     if (grid > a.total_items) grid = a.total_items > 0 ? a.total_items : 1;
     return sat::dispatch<sat::PREFILL>(a, D, Hq / Hkv, Hkv, (int)grid, s);
 }
@@ -374,7 +383,8 @@ cudaError_t launch_split_decode(const uint16_t *q, const uint16_t *k, const uint
     a.chunk = (n_entries + nsplit - 1) / nsplit;
     a.scale_log2 = scale * sat::LOG2E; a.o = o; a.lse = lse; a.part = part;
     a.status = status; a.total_items = (int64_t)B * nsplit;
-    int64_t grid = a.total_items < (int64_t)num_sms * 2 ? a.total_items : (int64_t)num_sms * 2;
+    const int64_t slots = (int64_t)num_sms * sat::Ring<sat::SPLIT>::CTAS;
+    int64_t grid = a.total_items < slots ? a.total_items : slots;
     cudaError_t e = sat::dispatch<sat::SPLIT>(a, D, Hq / Hkv, Hkv, (int)(grid > 0 ? grid : 1), s);
     if (e != cudaSuccess) return e;
     const int64_t n = (int64_t)B * Hq * D;
