@@ -143,17 +143,26 @@ __global__ void __launch_bounds__(THREADS, Ring<MODE>::CTAS) sparse_attn_kernel(
         __syncthreads();
 
         const int n_stage = (n_ent + C::NBS - 1) / C::NBS;
+        // TPB threads copy one block: thread li of block bi takes chunks
+        // li + TPB * k of the block's 4 key rows (block index read once)
+        constexpr int TPB = THREADS / C::NBS;
+        constexpr int MR = C::CHR / TPB;  // passes per key row
+        static_assert(TPB * C::NBS == THREADS && MR * TPB == C::CHR, "copy split");
+        const int bi = tid / TPB, li = tid % TPB;
         auto load_stage = [&](int s) {
             if (s < n_stage) {
                 uint8_t *dk = smem + (s % STAGES) * C::STAGE_BYTES;
                 uint8_t *dv = dk + C::STAGE_K;
-                for (int i = tid; i < C::KS * C::CHR; i += THREADS) {
-                    const int kk = i / C::CHR, ch = i % C::CHR;
-                    const int ent = s * C::NBS + (kk >> 2);
-                    const int j = ent < n_ent ? s_blk[ent] : -1;
-                    const int64_t u = (int64_t)j * 4 + (kk & 3);
-                    const bool ok = j >= 0 && u <= p;
-                    const int64_t off = ok ? u * (HKV * D) + ch * 8 : 0;
+                const int ent = s * C::NBS + bi;
+                const int j = ent < n_ent ? s_blk[ent] : -1;
+                const int64_t u0 = (int64_t)j * 4;
+#pragma unroll
+                for (int k = 0; k < 4 * MR; ++k) {
+                    const int r = k / MR;                    // token of the block
+                    const int ch = li + TPB * (k % MR);      // 16-byte chunk of its key row
+                    const int kk = bi * 4 + r;
+                    const bool ok = j >= 0 && u0 + r <= p;
+                    const int64_t off = ok ? (u0 + r) * (HKV * D) + ch * 8 : 0;
                     // chunk ch of the key row = head ch / (D/8), dim chunk ch % (D/8)
                     const int hh = ch / (D / 8), dc = ch % (D / 8);
                     const int dst = kk * C::ROW + hh * D * 2 + ((dc ^ (kk & 7)) * 16);
