@@ -62,6 +62,9 @@ constexpr int MAX_GRID = 160;
 template <int HI, int DI>
 struct L {
     static constexpr int NCOL = HI == 1 ? 128 : 256;  // MMA N
+    // two accumulator buffers; TMEM is allocated in powers of two columns
+    static constexpr int TMEM_COLS = 2 * NCOL <= 128 ? 128 : 2 * NCOL <= 256 ? 256 : 512;
+    static_assert(2 * NCOL <= 512, "TMEM");
     static constexpr int QT = NCOL / HI;              // queries per tile
     static constexpr int QPT = NCOL / 4 / HI;         // queries per epilogue thread
     static constexpr int ROWB = DI * 2;               // 64 or 128 bytes (= swizzle width)
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         *overflow = 0;
         sm100::fence_mbar_init();
     }
-    if (warp == 1) sm100::tmem_alloc(tmem_slot, 2 * NCOL);
+    if (warp == 1) sm100::tmem_alloc(tmem_slot, Lx::TMEM_COLS);
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
@@ -554,7 +557,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     if (warp == 1) {
         sm100::tc_fence_after();
-        sm100::tmem_dealloc(tmem_base, 2 * L<HI, DI>::NCOL);
+        sm100::tmem_dealloc(tmem_base, L<HI, DI>::TMEM_COLS);
     }
 }
 
