@@ -52,12 +52,13 @@ constexpr int STAGES = 4;
 constexpr int EPI_WARPS = 16;    // 4 per TMEM lane quarter
 constexpr int SEL_WARPS = 8;     // epilogue warps that also run the selections
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
-constexpr int CAP = 2048;        // candidate-list capacity per query (workspace)
+constexpr int CAP = 4096;        // candidate-list capacity per query (workspace)
 constexpr int SELBUF = 1024;     // per selecting warp, u64 keys in shared memory
-constexpr int CHECK_EVERY = 8;   // pass-2 tiles between list-capacity checks
+constexpr int CHECK_EVERY = 16;  // pass-2 tiles between list-capacity checks
 constexpr int MAX_GROUPS = 8;    // group maxima per block lane and query
 constexpr int MAX_KEEP = 511;
 constexpr int MAX_GRID = 160;
+constexpr int STG_ENT = 128;     // staged pass-2 survivors per epilogue warp
 
 template <int HI, int DI>
 struct L {
@@ -79,7 +80,9 @@ struct L {
     static constexpr int OFF_THR = OFF_W + QT * 16;
     static constexpr int OFF_C = OFF_THR + QT * 4;
     static constexpr int OFF_CNT = OFF_C + QT * 4;
-    static constexpr int OFF_BAR = OFF_CNT + QT * 4;
+    static constexpr int OFF_STGK = OFF_CNT + QT * 4;           // staged keys, per warp
+    static constexpr int OFF_STGX = OFF_STGK + EPI_WARPS * STG_ENT * 8;  // their query
+    static constexpr int OFF_BAR = OFF_STGX + EPI_WARPS * STG_ENT;
     static constexpr int NBAR = 2 * STAGES + 9;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
@@ -423,6 +426,22 @@ __global__ void __launch_bounds__(THREADS, 1)
             // this warp's survivor scores, [query x][lane]: the selection buffers
             // are idle during pass 2 (16 warps x QPT x 32 floats fit in them)
             float *scw = reinterpret_cast<float *>(sm + Lx::OFF_BUF) + e * (QPT * 32);
+            // survivors are staged per warp in shared memory (no atomic on the
+            // way) and moved to the query lists in batches, one entry per lane
+            uint64_t *stg_key = reinterpret_cast<uint64_t *>(sm + Lx::OFF_STGK) + e * STG_ENT;
+            uint8_t *stg_x = sm + Lx::OFF_STGX + e * STG_ENT;
+            int stg_n = 0;  // warp-uniform
+            auto append = [&](int x, uint64_t key) {
+                const int pos = atomicAdd(&s_cnt[q0 + x], 1);
+                if (pos < CAP) lists[(size_t)(q0 + x) * CAP + pos] = key;
+                if (pos == CAP - CHECK_EVERY * MB) *overflow = 1;
+            };
+            auto flush = [&]() {
+                __syncwarp();
+                for (int i = lane; i < stg_n; i += 32) append(stg_x[i], stg_key[i]);
+                __syncwarp();
+                stg_n = 0;
+            };
             for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
                 const int tb = it & 1;
                 sm100::mbar_wait(&tfull[tb], (it >> 1) & 1, abort_flag, a.wait_limit, a.ws);
@@ -454,19 +473,46 @@ __global__ void __launch_bounds__(THREADS, 1)
                 sm100::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) sm100::mbar_arrive(&tempty[tb]);
-                while (hit) {  // rare: about one survivor per 20 (thread, tile)
-                    const int b = 31 - __clz(hit);
-                    hit &= ~(1u << b);
-                    const int x = QPT - 1 - b;
-                    if (tail && j >= s_c[q0 + x]) continue;
-                    const int pos = atomicAdd(&s_cnt[q0 + x], 1);
-                    if (pos < CAP)
-                        lists[(size_t)(q0 + x) * CAP + pos] = idx::make_key(scw[x * 32 + lane], j);
-                    if (pos == CAP - CHECK_EVERY * MB) *overflow = 1;
+                if (tail) {  // blocks past a query's causal limit drop out
+                    uint32_t vm = 0;
+#pragma unroll
+                    for (int x = 0; x < QPT; ++x) vm = (vm << 1) | (uint32_t)(j < s_c[q0 + x]);
+                    hit &= vm;
+                }
+                if (__any_sync(0xffffffffu, hit != 0)) {  // most tiles at long range
+                    const int nl = __popc(hit);
+                    int incl = nl;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+                        if (lane >= off) incl += y;
+                    }
+                    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+                    if (stg_n + tot > STG_ENT) flush();
+                    if (tot > STG_ENT) {  // only with heavy ties: append directly
+                        while (hit) {
+                            const int b = 31 - __clz(hit);
+                            hit &= ~(1u << b);
+                            const int x = QPT - 1 - b;
+                            append(x, idx::make_key(scw[x * 32 + lane], j));
+                        }
+                    } else {
+                        int o = stg_n + incl - nl;
+                        while (hit) {
+                            const int b = 31 - __clz(hit);
+                            hit &= ~(1u << b);
+                            const int x = QPT - 1 - b;
+                            stg_key[o] = idx::make_key(scw[x * 32 + lane], j);
+                            stg_x[o] = (uint8_t)x;
+                            ++o;
+                        }
+                        stg_n += tot;
+                    }
                 }
                 // lists are checked every CHECK_EVERY tiles: a list below
                 // CAP - CHECK_EVERY * MB at a check cannot overflow before the next
                 if ((kt + 1) % CHECK_EVERY != 0 && kt + 1 != g.n_kt) continue;
+                flush();
                 epi_sync();
                 if (*overflow) {  // uniform: read after the barrier, set only before it
                     if (selw) {
