@@ -510,6 +510,8 @@ cudaError_t launch_index_topk_decode(const uint16_t *q_idx, const float *w, cons
                                      const int32_t *seqlens, int B, int64_t n_blocks, int Hi,
                                      int Di, int kb, int32_t *sel, float *sel_score, void *ws,
                                      int num_sms, cudaStream_t s) {
+    if (n_blocks == 0)  // every cache shorter than one block: nothing to score
+        return launch_own_block_only(nullptr, seqlens, B, 1, 0, kb, sel, sel_score, ws, s);
 #define QSA_DEC(HI_, DI_)          \
     if (Hi == HI_ && Di == DI_)    \
         return launch_dec<HI_, DI_>(q_idx, w, kp, seqlens, B, n_blocks, kb, sel, sel_score, ws, \

@@ -683,6 +683,9 @@ cudaError_t launch_index_topk_tc(const uint16_t *q_idx, const float *w, const ui
                                  const int64_t *q_pos0, int B, int64_t Tq, int64_t n_blocks,
                                  int Hi, int Di, int kb, int32_t *sel, float *sel_score, void *ws,
                                  int num_sms, cudaStream_t s) {
+    if (Tq == 0) return cudaSuccess;
+    if (n_blocks == 0)  // no complete block: nothing to score
+        return launch_own_block_only(q_pos0, nullptr, B, Tq, 0, kb, sel, sel_score, ws, s);
 #define QSA_ITC(HI_, DI_)        \
     if (Hi == HI_ && Di == DI_)  \
         return itc::launch<HI_, DI_>(q_idx, w, kp, q_pos0, B, Tq, n_blocks, kb, sel, sel_score, \

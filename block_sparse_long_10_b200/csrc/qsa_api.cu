@@ -146,7 +146,7 @@ qsa_status_t qsa_index_topk(const qsa_bf16_t *q_idx, const float *w, const qsa_b
         budget % r != 0)
         return QSA_ERR_INVALID_ARG;
     if (Tq == 0) return QSA_OK;
-    if (!q_idx || !w || !k_pooled || !sel) return QSA_ERR_INVALID_ARG;
+    if (!q_idx || !w || (!k_pooled && n_blocks > 0) || !sel) return QSA_ERR_INVALID_ARG;
     if (!q_pos0 && (Tq - 1) / r > n_blocks) return QSA_ERR_INVALID_ARG;
     const int kb = budget / r;
     if (r != 4 || !supported_indexer(Hi, Di) || kb - 1 > qsa::index_tc_max_keep())
@@ -174,7 +174,8 @@ qsa_status_t qsa_index_topk_decode(const qsa_bf16_t *q_idx, const float *w,
                                    void *stream) {
     if (B < 1 || n_blocks < 0 || Hi < 1 || Di < 1 || r < 1 || budget < r || budget % r != 0)
         return QSA_ERR_INVALID_ARG;
-    if (!q_idx || !w || !k_pooled || !seqlens || !sel) return QSA_ERR_INVALID_ARG;
+    if (!q_idx || !w || (!k_pooled && n_blocks > 0) || !seqlens || !sel)
+        return QSA_ERR_INVALID_ARG;
     const int kb = budget / r;
     if (r != 4 || !supported_indexer(Hi, Di) || kb - 1 > qsa::index_tc_max_keep() ||
         qsa::index_decode_merge_cap(n_blocks, kb) < 0)
@@ -196,11 +197,11 @@ qsa_status_t qsa_sparse_attn_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k,
                                      const int64_t *q_pos0, int B, int64_t Tq, int64_t Tk,
                                      int Hq, int Hkv, int D, int r, int budget, float scale,
                                      qsa_bf16_t *o, float *lse, void *stream) {
-    if (B < 1 || Tq < 0 || Tk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || D < 1 || r < 1 ||
+    if (B < 1 || Tq < 0 || Tk < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || D < 1 || r < 1 ||
         budget < r || budget % r != 0 || !(scale == scale))
         return QSA_ERR_INVALID_ARG;
     if (Tq == 0) return QSA_OK;
-    if (!q || !k || !v || !sel || !o) return QSA_ERR_INVALID_ARG;
+    if (Tk < 1 || !q || !k || !v || !sel || !o) return QSA_ERR_INVALID_ARG;
     if (!q_pos0 && Tq > Tk) return QSA_ERR_INVALID_ARG;
     const int kb = budget / r;
     if (r != 4 || !supported_attn(Hq, Hkv, D) || kb > 1024) return QSA_ERR_UNSUPPORTED_SHAPE;

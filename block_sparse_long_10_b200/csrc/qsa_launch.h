@@ -20,6 +20,11 @@ cudaError_t launch_pool(const uint16_t *k_idx, int B, int64_t T, int Di, int64_t
 int index_tc_grid(int B, int64_t Tq, int Hi);
 size_t index_tc_ws_bytes(int B, int64_t Tq, int Hi);
 int index_tc_max_keep();
+// Every query keeps only its own block (n_blocks == 0: no complete block yet).
+// q_pos0/seqlens as in the indexers (seqlens != nullptr: decode, Tq = 1).
+cudaError_t launch_own_block_only(const int64_t *q_pos0, const int32_t *seqlens, int B, int64_t Tq,
+                                  int64_t n_blocks, int kb, int32_t *sel, float *sel_score,
+                                  void *status, cudaStream_t s);
 cudaError_t launch_index_topk_tc(const uint16_t *q_idx, const float *w, const uint16_t *kp,
                                  const int64_t *q_pos0, int B, int64_t Tq, int64_t n_blocks,
                                  int Hi, int Di, int kb, int32_t *sel, float *sel_score, void *ws,

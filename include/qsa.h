@@ -96,7 +96,8 @@ QSA_API qsa_status_t qsa_pool(const qsa_bf16_t *k_idx, int B, int64_t T, int Di,
  * padded with -1, kb = budget / r entries per query.
  *   q_idx     [B, Tq, Hi, Di] bf16
  *   w         [B, Tq, Hi] fp32 per-token head weights
- *   k_pooled  [B, n_blocks, Di] bf16
+ *   k_pooled  [B, n_blocks, Di] bf16 (may be NULL when n_blocks == 0: every
+ *             query then keeps its own block only)
  *   q_pos0    [B] int64 device array, or NULL
  *   sel       [B, Tq, kb] int32 (output)
  *   sel_score [B, Tq, kb] fp32 (output, may be NULL): the score of each kept
@@ -104,7 +105,7 @@ QSA_API qsa_status_t qsa_pool(const qsa_bf16_t *k_idx, int B, int64_t T, int Di,
  *   ws        device workspace of at least qsa_index_topk_workspace_size(...)
  *             bytes; its first 256 bytes hold the device status word
  * A position whose floor(p / r) exceeds n_blocks is clamped to n_blocks and
- * recorded as QSA_ERR_DEVICE in the status word.
+ * recorded as QSA_ERR_DEVICE in the status word.  Tq == 0 is a no-op.
  */
 QSA_API size_t qsa_index_topk_workspace_size(int B, int64_t Tq, int64_t n_blocks, int Hi,
                                      int Di, int r, int budget);
@@ -119,7 +120,8 @@ QSA_API qsa_status_t qsa_index_topk(const qsa_bf16_t *q_idx, const float *w,
  * same scores, ranking and output as qsa_index_topk with Tq = 1, but the
  * candidates of each sequence are split across many CTAs and merged, so a
  * batch of 64 sequences fills the GPU.
- *   q_idx [B, Hi, Di] bf16, w [B, Hi] fp32, k_pooled [B, n_blocks, Di] bf16,
+ *   q_idx [B, Hi, Di] bf16, w [B, Hi] fp32, k_pooled [B, n_blocks, Di] bf16
+ *   (may be NULL when n_blocks == 0),
  *   seqlens [B] int32 device array (1 <= seqlens[b] and
  *   floor((seqlens[b] - 1) / r) <= n_blocks, else clamped and recorded as
  *   QSA_ERR_DEVICE), sel [B, kb] int32, sel_score [B, kb] fp32 (nullable).

@@ -83,6 +83,7 @@ def test_index_topk_validation(lib):
     assert call(args(budget=2047)) == INVALID
     assert call(args(B=0)) == INVALID
     assert call(args(q=_nullp())) == INVALID
+    assert call(args(kp=_nullp())) == INVALID           # pooled keys needed when N > 0
     assert call(args(N=100)) == INVALID                 # queries beyond the pooled keys
     assert call(args(Hi=3)) == UNSUPPORTED
     assert call(args(Di=48)) == UNSUPPORTED
@@ -108,6 +109,8 @@ def test_attention_validation(lib):
     assert sp(Tq=65) == INVALID                        # queries beyond K/V without q_pos0
     assert sp(budget=8192) == UNSUPPORTED               # kb > 1024
     assert sp(Tq=0) == OK
+    assert sp(Tq=0, Tk=0) == OK                        # empty sequence: no-op
+    assert sp(Tk=0) == INVALID
     nan = ctypes.c_float(float("nan"))
     assert lib.qsa_dense_gqa_prefill(f, f, f, 1, 64, 16, 2, 128, nan, f, None, s) == INVALID
     assert lib.qsa_dense_gqa_prefill(f, f, f, 1, 64, 16, 2, 80, ctypes.c_float(.1), f, None,
