@@ -186,10 +186,15 @@ QSA_DEVICE uint64_t *warp_radix_sort_hi32(uint64_t *buf, uint64_t *tmp, int m, i
             const bool v = i < m;
             const uint64_t k = v ? buf[i] : 0ull;
             const uint32_t d = (uint32_t)(k >> sh) & 255u;
-            const uint32_t act = __ballot_sync(0xffffffffu, v);
-            uint32_t peers = 0, base = 0;
+            // lanes holding the same digit: one ballot per digit bit
+            uint32_t peers = __ballot_sync(0xffffffffu, v);
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const uint32_t bal = __ballot_sync(0xffffffffu, (d >> b) & 1u);
+                peers &= ((d >> b) & 1u) ? bal : ~bal;
+            }
+            uint32_t base = 0;
             if (v) {
-                peers = __match_any_sync(act, d);
                 base = hist[d];
                 tmp[base + __popc(peers & lt)] = k;
             }
