@@ -325,10 +325,9 @@ __global__ void __launch_bounds__(SEL_THREADS)
         if (n > K && G >= K) {
             for (int i = tid; i < G; i += SEL_THREADS) list[i] = ((uint64_t)gm[i] << 32) | (uint32_t)i;
             __syncthreads();
-            if (tid < 32) {  // small array: one warp, no block barriers
-                const uint64_t kth = idx::warp_kth_largest(list, G, K, hist, tid);
-                if (tid == 0) s_theta = key_score((uint32_t)(kth >> 32));
-            }
+            const uint64_t kth =
+                block_kth_largest([&](int i) { return list[i]; }, G, K, hist, sh, red);
+            if (tid == 0) s_theta = key_score((uint32_t)(kth >> 32));
         }
         if (tid == 0) s_cnt = 0;
         __syncthreads();
@@ -355,16 +354,8 @@ __global__ void __launch_bounds__(SEL_THREADS)
         const int cnt = s_cnt;
         __syncthreads();
         uint64_t kth = 0;
-        __shared__ uint64_t s_kth;
         if (cnt <= LIST_CAP) {
-            if (cnt > K) {
-                if (tid < 32) {
-                    const uint64_t k2 = idx::warp_kth_largest(list, cnt, K, hist, tid);
-                    if (tid == 0) s_kth = k2;
-                }
-                __syncthreads();
-                kth = s_kth;
-            }
+            if (cnt > K) kth = block_kth_largest([&](int i) { return list[i]; }, cnt, K, hist, sh, red);
         } else {  // many ties at theta: exact select over every score
             kth = block_kth_largest([&](int i) { return make_key(sc[i], i); }, n, K, hist, sh,
                                     red);
