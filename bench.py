@@ -342,9 +342,24 @@ def kernel_report(w, kern_ms, peaks):
     return rep, wk
 
 
+# DRAM bytes (read + write) per launch, from one single-pass ncu capture of the
+# same command's kernels (profiles/launches_prefill-1m.md gives the command and
+# the counters):  ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
+# dram__bytes_write.sum --clock-control none -k regex:"idx_tc|sparse_attn"
+# -s 4 -c 2 python bench.py --steps 1 --warmup 3 --no-extra --no-dense
+# --no-e2e --no-cpu.  Keyed by (workload, kernel); must be re-taken (or
+# removed) whenever that kernel changes.
+MEASURED_TRAFFIC = {
+    ("prefill-1m", "index_topk"): 3.81e9 + 12.00e9,
+    ("prefill-1m", "sparse_attn"): 552.82e9 + 4.30e9,
+}
+
+
 def dominant_roofline(w, kern_ms, peaks, traffic=None):
     wk = prefill_work(w)
     name = max(kern_ms, key=kern_ms.get)
+    if traffic is None:
+        traffic = MEASURED_TRAFFIC.get((w.name, name))
     s = kern_ms[name] / 1e3
     if name == "index_topk":
         r = roof(wk["index_flops"] / s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s",

@@ -74,8 +74,10 @@ bool supported_indexer(int Hi, int Di) {
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// About one wave of slices (2 CTAs per SM on 148 SMs ~ 296 slots): at 64
+// sequences, 4 slices of 128 blocks each.
 int sparse_decode_nsplit(int B, int kb) {
-    int ns = (int)cdiv(512, B > 0 ? B : 1);
+    int ns = (int)cdiv(256, B > 0 ? B : 1);
     int max_ns = kb / 16 > 1 ? kb / 16 : 1;
     if (ns > max_ns) ns = max_ns;
     return ns < 1 ? 1 : ns;
