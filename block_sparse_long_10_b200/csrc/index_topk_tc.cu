@@ -18,8 +18,9 @@
 //               issues D[128 blocks, NCOL columns] = Kp_tile x Q_tile^T as
 //               Di/16 tcgen05.mma (bf16 in, fp32 in TMEM), double-buffered;
 //   warps 2-17  epilogue: TMEM lane = block, so each thread reads one block's
-//               scores for a quarter of the columns (32x32b loads) and forms
-//               the ReLU-weighted head sum in registers.
+//               scores for a quarter of the columns (32x32b loads, 16 columns
+//               at a time) and forms the ReLU-weighted head sum in registers,
+//               two heads per packed f32x2 multiply-add.
 // Each query tile is swept twice (the pooled keys stay in L2):
 //   pass 1  every thread keeps, per query, the maximum score of its block
 //           lane over groups of R consecutive tiles (at most 8 groups, so at
@@ -30,7 +31,11 @@
 //   pass 2  the same scores, recomputed bit for bit, are filtered by
 //           s >= theta and appended (64-bit key: order-preserving score bits
 //           above the complemented block index) to the query's list in the
-//           workspace.  Every top-(kb-1) candidate has s >= theta.
+//           workspace.  Every top-(kb-1) candidate has s >= theta.  The test
+//           is branch-free (a bit mask per thread, the survivor's score parked
+//           in shared memory); survivors are staged per warp in shared memory
+//           and moved to the lists in batches, and the lists are checked for
+//           capacity every CHECK_EVERY tiles.
 // Finalisation (per query): exact radix select of the list's kb - 1 best
 // keys in shared memory, stable radix sort by block id, own block appended.
 // A list that would overflow (only with heavily tied scores) is cut to its
