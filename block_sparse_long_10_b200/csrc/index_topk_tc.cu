@@ -12,7 +12,7 @@
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: the CTA's query tile (NCOL (query, head) rows,
-//               double-buffered) and a 4-stage ring of 128-block pooled-key
+//               double-buffered) and a 3-stage ring of 128-block pooled-key
 //               tiles, 128/64-byte swizzled;
 //   warp 1      TMEM owner and MMA issuer: per pooled-key tile one thread
 //               issues D[128 blocks, NCOL columns] = Kp_tile x Q_tile^T as
