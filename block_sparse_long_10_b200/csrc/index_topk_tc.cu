@@ -676,12 +676,6 @@ size_t index_tc_ws_bytes(int B, int64_t Tq, int Hi) {
     return itc::ws_bytes<4>(B, Tq);
 }
 
-int index_tc_grid(int B, int64_t Tq, int Hi) {
-    if (Hi == 1) return itc::grid_for<1>(B, Tq);
-    if (Hi == 2) return itc::grid_for<2>(B, Tq);
-    return itc::grid_for<4>(B, Tq);
-}
-
 int index_tc_max_keep() { return itc::MAX_KEEP; }
 
 cudaError_t launch_index_topk_tc(const uint16_t *q_idx, const float *w, const uint16_t *kp,

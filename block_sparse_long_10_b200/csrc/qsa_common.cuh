@@ -14,7 +14,6 @@ namespace qsa {
 // Workspace header: the sticky status word lives at byte 0, per-call scratch
 // counters start at byte 64; kernel data starts after the first 256 bytes.
 constexpr size_t kWsHeader = 256;
-constexpr size_t kWsCounters = 64;
 
 QSA_DEVICE void record_status(void *ws, int code) {
     if (ws) atomicCAS(reinterpret_cast<int *>(ws), 0, code);

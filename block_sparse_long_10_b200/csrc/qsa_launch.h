@@ -17,7 +17,6 @@ bool tensor_map_2d_bf16(CUtensorMap_st *out, const void *base, uint64_t rows, ui
 cudaError_t launch_pool(const uint16_t *k_idx, int B, int64_t T, int Di, int64_t j0,
                         int64_t j1, uint16_t *kp, cudaStream_t s, int num_sms);
 
-int index_tc_grid(int B, int64_t Tq, int Hi);
 size_t index_tc_ws_bytes(int B, int64_t Tq, int Hi);
 int index_tc_max_keep();
 // Every query keeps only its own block (n_blocks == 0: no complete block yet).

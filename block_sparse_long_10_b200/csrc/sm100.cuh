@@ -135,7 +135,6 @@ QSA_DEVICE void mma_commit(uint64_t *bar) {
             smem_u32(bar))
         : "memory");
 }
-QSA_DEVICE void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
 // 32 lanes x 16 consecutive fp32 columns: thread i gets lane (base + i).  The
 // wait is in the same statement, so the registers are complete when it returns.

@@ -128,21 +128,6 @@ QSA_DEVICE int warp_compact_ge(uint64_t *buf, int n, uint64_t kth, int lane) {
     return base;
 }
 
-// Stable copy of the keys >= kth from src to dst; returns how many.
-QSA_DEVICE int warp_copy_ge(uint64_t *dst, const uint64_t *src, int n, uint64_t kth, int lane) {
-    int base = 0;
-    for (int i0 = 0; i0 < n; i0 += 32) {
-        const int i = i0 + lane;
-        const uint64_t k = (i < n) ? src[i] : 0ull;
-        const bool keep = (i < n) && (k >= kth);
-        const uint32_t m = __ballot_sync(0xffffffffu, keep);
-        if (keep) dst[base + __popc(m & ((1u << lane) - 1u))] = k;
-        base += __popc(m);
-    }
-    __syncwarp();
-    return base;
-}
-
 // Stable LSD radix sort (8-bit digits) of m <= 1024 keys by their high 32
 // bits, which hold values below 2^(8*passes).  Ping-pongs between buf and
 // tmp; returns the buffer that holds the result.
