@@ -12,7 +12,7 @@
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: the CTA's query tile (NCOL (query, head) rows,
-//               double-buffered) and a 3-stage ring of 128-block pooled-key
+//               double-buffered) and a 4-stage ring of 128-block pooled-key
 //               tiles, 128/64-byte swizzled;
 //   warp 1      TMEM owner and MMA issuer: per pooled-key tile one thread
 //               issues D[128 blocks, NCOL columns] = Kp_tile x Q_tile^T as
@@ -53,9 +53,9 @@ namespace qsa {
 namespace itc {
 
 constexpr int MB = 128;          // pooled blocks per tile = MMA M = TMEM lanes
-constexpr int STAGES = 3;
+constexpr int STAGES = 4;
 constexpr int EPI_WARPS = 16;    // 4 per TMEM lane quarter
-constexpr int SEL_WARPS = 10;    // epilogue warps that also run the selections
+constexpr int SEL_WARPS = 8;     // epilogue warps that also run the selections
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr int CAP = 4096;        // candidate-list capacity per query (workspace)
 constexpr int SELBUF = 1024;     // per selecting warp, u64 keys in shared memory

@@ -11,8 +11,8 @@
 
 namespace qsa {
 
-// Workspace header: the sticky status word lives at byte 0, per-call scratch
-// counters start at byte 64; kernel data starts after the first 256 bytes.
+// Workspace header: the sticky status word lives at byte 0; kernel data starts
+// after the first 256 bytes.
 constexpr size_t kWsHeader = 256;
 
 QSA_DEVICE void record_status(void *ws, int code) {

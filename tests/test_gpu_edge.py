@@ -111,3 +111,43 @@ def test_decode_caches_shorter_than_one_block():
     assert st == (0, 0)
     assert (sel[:, 0] == 0).all() and (sel[:, 1:] == -1).all()
     _check_decode_rows(w, x, kp, sel, sc, o, lse, range(w.B))
+
+
+def test_chunked_prefill_equals_one_shot():
+    """Prefill in chunks (q_pos0 = chunk start, pooling only the blocks that each
+    chunk completes) gives the same pooled keys and selections, and bit-identical
+    outputs, as one call over the whole sequence."""
+    w = synth.Workload("chunks", "prefill", 1, 3001, 8, 2, 128, 4, 64, 4, 256, 61, 4)
+    x = synth.make_prefill(w, DEV)
+    kp1, sel1, sc1, o1, lse1 = _qsa_prefill(x, w)
+    T, N = w.T, w.T // w.r
+    kp = torch.zeros(1, N, w.Di, dtype=BF, device=DEV)
+    sel = torch.empty(1, T, w.kb, dtype=torch.int32, device=DEV)
+    o = torch.empty_like(x["q"])
+    lse = torch.empty(1, T, w.Hq, dtype=torch.float32, device=DEV)
+    bounds = [0, 1000, 2203, T]
+    done = 0
+    for c0, c1 in zip(bounds[:-1], bounds[1:]):
+        nb = c1 // w.r
+        qsa.qsa_pool(x["k_idx"], kp, w.r, blk_begin=done, blk_end=nb)
+        done = nb
+        pos0 = torch.tensor([c0], dtype=torch.int64, device=DEV)
+        tq = c1 - c0
+        selc = torch.empty(1, tq, w.kb, dtype=torch.int32, device=DEV)
+        ws = qsa.workspace(qsa.qsa_index_topk_workspace_size(1, tq, nb, w.Hi, w.Di, w.r, w.budget))
+        qsa.qsa_index_topk(x["q_idx"][:, c0:c1].contiguous(), x["w"][:, c0:c1].contiguous(),
+                           kp[:, :nb], selc, ws, w.r, w.budget, q_pos0=pos0)
+        oc = torch.empty(1, tq, w.Hq, w.D, dtype=BF, device=DEV)
+        lc = torch.empty(1, tq, w.Hq, dtype=torch.float32, device=DEV)
+        qsa.qsa_sparse_attn_prefill(x["q"][:, c0:c1].contiguous(), x["k"][:, :c1].contiguous(),
+                                    x["v"][:, :c1].contiguous(), selc, oc, w.r, w.budget,
+                                    w.scale, q_pos0=pos0, lse=lc)
+        assert qsa.qsa_check_device_status(ws) == 0
+        sel[:, c0:c1] = selc
+        o[:, c0:c1] = oc
+        lse[:, c0:c1] = lc
+    torch.cuda.synchronize()
+    assert torch.equal(kp, kp1)
+    assert torch.equal(sel, sel1)
+    assert torch.equal(o.view(torch.int16), o1.view(torch.int16))
+    assert torch.equal(lse, lse1)
