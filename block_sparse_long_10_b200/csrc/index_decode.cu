@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(SEL_THREADS)
     decode_select_kernel(const float *__restrict__ scores, const uint32_t *__restrict__ gmax,
                          const int32_t *__restrict__ seqlens, int64_t n_blocks, int kb,
                          int nsplit, int32_t *__restrict__ sel, float *__restrict__ sel_score) {
+    griddep_wait();  // the scores and maxima of the scoring kernel
     extern __shared__ __align__(16) uint8_t smem[];
     uint64_t *list = reinterpret_cast<uint64_t *>(smem);  // [LIST_CAP] survivors
     uint64_t *kept = list + LIST_CAP;                      // [1024] kept keys
@@ -492,9 +493,9 @@ static cudaError_t launch_dec(const uint16_t *q_idx, const float *w, const uint1
     const int smem2 = (idd::LIST_CAP + 2048) * 8;
     e = ensure_smem(reinterpret_cast<const void *>(idd::decode_select_kernel), smem2);
     if (e != cudaSuccess) return e;
-    idd::decode_select_kernel<<<B, idd::SEL_THREADS, smem2, s>>>(scores, gmax, seqlens, n_blocks,
-                                                                  kb, ns, sel, sel_score);
-    return cudaGetLastError();
+    return launch_dependent(idd::decode_select_kernel, dim3(B), dim3(idd::SEL_THREADS),
+                            (size_t)smem2, s, scores, (const uint32_t *)gmax, seqlens, n_blocks,
+                            kb, ns, sel, sel_score);
 }
 
 cudaError_t launch_index_topk_decode(const uint16_t *q_idx, const float *w, const uint16_t *kp,

@@ -15,6 +15,11 @@ namespace qsa {
 // after the first 256 bytes.
 constexpr size_t kWsHeader = 256;
 
+// Kernels launched as programmatic dependents (launch_dependent) start while
+// the previous kernel in the stream drains; this waits until that kernel has
+// completed and its memory is visible.  A no-op for an ordinary launch.
+QSA_DEVICE void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 QSA_DEVICE void record_status(void *ws, int code) {
     if (ws) atomicCAS(reinterpret_cast<int *>(ws), 0, code);
 }

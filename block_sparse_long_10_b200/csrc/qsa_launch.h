@@ -11,6 +11,25 @@ namespace qsa {
 
 // Host caches (host_util.cu).
 cudaError_t ensure_smem(const void *kern, int bytes);
+
+// Launch `kern` as a programmatic dependent of the previous kernel in `s`:
+// its launch overlaps that kernel's tail; the kernel itself must call
+// griddep_wait() before it reads anything the previous kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 bool tensor_map_2d_bf16(CUtensorMap_st *out, const void *base, uint64_t rows, uint32_t cols,
                         uint32_t box_rows);
 

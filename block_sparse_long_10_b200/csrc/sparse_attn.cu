@@ -82,6 +82,7 @@ struct Args {
 
 template <int D, int G, int HKV, int MODE>
 __global__ void __launch_bounds__(THREADS, Ring<MODE>::CTAS) sparse_attn_kernel(const Args a) {
+    griddep_wait();  // the selection (and partial buffers) of the previous kernel
     constexpr int STAGES = Ring<MODE>::STAGES;
     using C = Cfg<D, HKV, STAGES>;
     constexpr int KSTEP = D / 16;
@@ -316,6 +317,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const float *__restr
                                                             int B, int Hq, int nsplit,
                                                             uint16_t *__restrict__ o,
                                                             float *__restrict__ lse) {
+    griddep_wait();  // the split partials
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= (int64_t)B * Hq * D) return;
     const int d = (int)(i % D);
@@ -344,8 +346,7 @@ static cudaError_t launch_sat(const Args &a, int grid, cudaStream_t s) {
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
     if (e != cudaSuccess) return e;
     if (a.total_items == 0) return cudaSuccess;
-    kern<<<grid, THREADS, C::BYTES, s>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3(grid), dim3(THREADS), (size_t)C::BYTES, s, a);
 }
 
 template <int MODE>
@@ -398,13 +399,12 @@ cudaError_t launch_split_decode(const uint16_t *q, const uint16_t *k, const uint
     if (e != cudaSuccess) return e;
     const int64_t n = (int64_t)B * Hq * D;
     if (n == 0) return cudaSuccess;
+    const dim3 cgrid((unsigned)((n + 255) / 256));
     if (D == 64)
-        sat::split_combine_kernel<64><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, B, Hq,
-                                                                                nsplit, o, lse);
-    else
-        sat::split_combine_kernel<128><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, B, Hq,
-                                                                                 nsplit, o, lse);
-    return cudaGetLastError();
+        return launch_dependent(sat::split_combine_kernel<64>, cgrid, dim3(256), 0, s,
+                                (const float *)part, B, Hq, nsplit, o, lse);
+    return launch_dependent(sat::split_combine_kernel<128>, cgrid, dim3(256), 0, s,
+                            (const float *)part, B, Hq, nsplit, o, lse);
 }
 
 }  // namespace qsa
