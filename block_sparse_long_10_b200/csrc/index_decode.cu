@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(THREADS, 3)
                         const float *__restrict__ w, const int32_t *__restrict__ seqlens,
                         int64_t n_blocks, int nsplit, int n_items, float *__restrict__ scores,
                         uint32_t *__restrict__ gmax, void *ws) {
+    griddep_wait();  // inputs (pooled keys, queries, lengths) of earlier kernels
     constexpr int ROWB = DI * 2, CH = DI / 8, KSTEPS = DI / 16;
     constexpr int TILE = NB * ROWB;
     extern __shared__ uint8_t smem_raw[];
@@ -486,9 +487,8 @@ static cudaError_t launch_dec(const uint16_t *q_idx, const float *w, const uint1
     if (e != cudaSuccess) return e;
     const int n_items = B * ns;
     const int grid = n_items < 3 * sms ? n_items : 3 * sms;
-    k1<<<grid, idd::THREADS, smem1, s>>>(tm, q_idx, w, seqlens, n_blocks, ns, n_items, scores,
-                                         gmax, ws);
-    e = cudaGetLastError();
+    e = launch_dependent(k1, dim3(grid), dim3(idd::THREADS), (size_t)smem1, s, tm, q_idx, w,
+                         seqlens, n_blocks, ns, n_items, scores, gmax, ws);
     if (e != cudaSuccess) return e;
     const int smem2 = (idd::LIST_CAP + 2048) * 8;
     e = ensure_smem(reinterpret_cast<const void *>(idd::decode_select_kernel), smem2);
