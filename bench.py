@@ -350,8 +350,8 @@ def kernel_report(w, kern_ms, peaks):
 # --no-e2e --no-cpu.  Keyed by (workload, kernel); must be re-taken (or
 # removed) whenever that kernel changes.
 MEASURED_TRAFFIC = {
-    ("prefill-1m", "index_topk"): 3.87e9 + 12.01e9,
-    ("prefill-1m", "sparse_attn"): 559.62e9 + 4.30e9,
+    # ("prefill-1m", "index_topk"): re-take after the 32-bit bound selection
+    # (last capture, of the kernel before it: 3.87e9 + 12.01e9)
 }
 
 

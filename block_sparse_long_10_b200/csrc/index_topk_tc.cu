@@ -81,6 +81,8 @@ struct L {
     static constexpr int OFF_BUF = OFF_Q + 2 * Q_TILE;
     static constexpr int OFF_HIST = OFF_BUF + SEL_WARPS * SELBUF * 8;
     static_assert(EPI_WARPS * QPT * 32 * 4 <= SEL_WARPS * SELBUF * 8, "pass-2 score park");
+    static_assert(EPI_WARPS * MAX_GROUPS * MB * 4 <= SEL_WARPS * SELBUF * 8, "bound keys");
+    static_assert((EPI_WARPS - SEL_WARPS) * 256 * 4 <= EPI_WARPS * STG_ENT * 8, "bound hists");
     static constexpr int OFF_W = OFF_HIST + SEL_WARPS * 256 * 4;
     static constexpr int OFF_THR = OFF_W + QT * 16;
     static constexpr int OFF_C = OFF_THR + QT * 4;
@@ -403,18 +405,24 @@ __global__ void __launch_bounds__(THREADS, 1)
             epi_sync();
 
             // ---- theta: the (kb-1)-th largest group maximum --------------
-            if (selw) {
+            // every epilogue warp takes queries; the bound needs the score value
+            // only, so the keys are the 32-bit score keys (the selection
+            // buffers hold 16 x 1024 of them; warps past the selecting ones
+            // keep their histograms in the idle staging area)
+            {
+                uint32_t *kbuf = reinterpret_cast<uint32_t *>(sm + Lx::OFF_BUF) + e * (MAX_GROUPS * MB);
+                uint32_t *th_hist = selw ? hist
+                                         : reinterpret_cast<uint32_t *>(sm + Lx::OFF_STGK) +
+                                               (e - SEL_WARPS) * 256;
 #pragma unroll 1
-                for (int q = e; q < QT; q += SEL_WARPS) {
+                for (int q = e; q < QT; q += EPI_WARPS) {
                     float th = K > 0 ? -INFINITY : INFINITY;
                     const int G = n_groups * MB;
                     if (K > 0 && G >= K && g.t0 + q < a.Tq) {
                         const uint32_t *src = gmax_g + (size_t)q * (MAX_GROUPS * MB);
-                        for (int x = lane; x < G; x += 32)
-                            buf[x] = ((uint64_t)src[x] << 32) | (uint32_t)x;
+                        for (int x = lane; x < G; x += 32) kbuf[x] = src[x];
                         __syncwarp();
-                        const uint64_t kth = idx::warp_kth_largest(buf, G, K, hist, lane);
-                        th = key_score((uint32_t)(kth >> 32));
+                        th = key_score(idx::warp_kth_largest_u32(kbuf, G, K, th_hist, lane));
                     }
                     if (g.t0 + q >= a.Tq) th = INFINITY;   // padding queries keep nothing
                     if (lane == 0) s_thr[q] = th;

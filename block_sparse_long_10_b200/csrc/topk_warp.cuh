@@ -113,6 +113,87 @@ QSA_DEVICE uint64_t warp_kth_largest(const uint64_t *buf, int n, int K, uint32_t
     }
 }
 
+// The K-th largest of n 32-bit keys (1 <= K <= n; equal keys allowed: the
+// result is the K-th value counting multiplicity), same digit scheme.
+QSA_DEVICE uint32_t warp_kth_largest_u32(const uint32_t *buf, int n, int K, uint32_t *hist,
+                                         int lane) {
+    uint32_t mn = ~0u, mx = 0u;
+    for (int i = lane; i < n; i += 32) {
+        const uint32_t k = buf[i];
+        mn = k < mn ? k : mn;
+        mx = k > mx ? k : mx;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    if (mn == mx || K >= n) return mn;
+    if (K == 1) return mx;
+    int top = 31 - __clz((int)(mn ^ mx));
+    uint32_t prefix = top >= 31 ? 0u : (mn & (~0u << (top + 1)));
+    int want = K;
+#pragma unroll 1
+    for (;;) {
+        const int shift = top - 7;
+        const uint32_t hm = top >= 31 ? 0u : (~0u << (top + 1));
+        for (int i = lane; i < 256; i += 32) hist[i] = 0;
+        __syncwarp();
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t k = i < n ? buf[i] : 0u;
+            const bool m = i < n && (k & hm) == prefix;
+            const uint32_t d = (shift >= 0 ? (k >> shift) : (k << -shift)) & 255u;
+            hist_add(hist, d, m, lane);
+        }
+        __syncwarp();
+        uint32_t local[8], sum = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            local[b] = hist[lane * 8 + b];
+            sum += local[b];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+            if (lane + off < 32) incl += y;
+        }
+        uint32_t cum = incl - sum;
+        int found = -1, new_want = 0;
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int b = 7; b >= 0; --b) {
+            if (found < 0 && (int)cum < want && want <= (int)(cum + local[b])) {
+                found = lane * 8 + b;
+                new_want = want - (int)cum;
+                cnt = local[b];
+            }
+            cum += local[b];
+        }
+        const uint32_t ball = __ballot_sync(0xffffffffu, found >= 0);
+        const int src = __ffs(ball) - 1;
+        found = __shfl_sync(0xffffffffu, found, src);
+        want = __shfl_sync(0xffffffffu, new_want, src);
+        cnt = __shfl_sync(0xffffffffu, cnt, src);
+        prefix |= shift >= 0 ? ((uint32_t)found << shift) : ((uint32_t)found >> -shift);
+        __syncwarp();
+        if (shift <= 0) return prefix;
+        if ((int)cnt == want) {  // bucket kept whole: its minimum is the answer
+            const uint32_t m2 = ~0u << shift;
+            uint32_t bmin = ~0u;
+            for (int i = lane; i < n; i += 32) {
+                const uint32_t k = buf[i];
+                if ((k & m2) == prefix && k < bmin) bmin = k;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) bmin = min(bmin, __shfl_xor_sync(0xffffffffu, bmin, off));
+            return bmin;
+        }
+        top = shift - 1;
+    }
+}
+
 // Keep the keys >= kth (exactly K of them) at the front of buf; returns count.
 QSA_DEVICE int warp_compact_ge(uint64_t *buf, int n, uint64_t kth, int lane) {
     int base = 0;
