@@ -27,6 +27,7 @@ __all__ = [
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode_noalloc",
     "qsa_dense_gqa_prefill",
     "qsa_dense_gqa_decode", "qsa_dense_gqa_decode_workspace_size",
+    "qsa_index_distill", "qsa_index_distill_workspace_size",
     "qsa_check_device_status", "qsa_status_string", "qsa_version",
 ]
 
@@ -73,6 +74,9 @@ _SIGS = {
     "qsa_dense_gqa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "qsa_dense_gqa_decode": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _F,
                                   _VP, _VP, _VP, _SZ, _VP]),
+    "qsa_index_distill_workspace_size": (_SZ, [_I, _I64, _I, _I]),
+    "qsa_index_distill": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
+                               _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "qsa_check_device_status": (_I, [_VP, _VP]),
     "qsa_status_string": (ctypes.c_char_p, [_I]),
     "qsa_version": (ctypes.c_char_p, []),
@@ -289,6 +293,43 @@ def qsa_dense_gqa_decode(q, k_cache, v_cache, seqlens, o, ws, scale=None, lse=No
     scale = D ** -0.5 if scale is None else scale
     _call("qsa_dense_gqa_decode", _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), L, B,
           Hq, Hkv, D, scale, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream, q.device))
+
+
+# ----------------------------------------------------- indexer distillation --
+
+def qsa_index_distill_workspace_size(B, T, Hkv, r=4) -> int:
+    return _size("qsa_index_distill_workspace_size", B, T, Hkv, r)
+
+
+def qsa_index_distill(q, k, lse, q_idx, w, k_pooled, kl, dq_idx, dw, dk_pooled, ws, r=4,
+                      scale=None, dk_idx=None, stream=None):
+    """Stage-1 distillation loss and indexer gradients.
+
+    q [B,T,Hq,D], k [B,T,Hkv,D] bf16, lse [B,T,Hq] fp32 (dense attention's),
+    q_idx [B,T,Hi,Di] bf16, w [B,T,Hi] fp32, k_pooled [B,T//r,Di] bf16 ->
+    kl [B,T], dq_idx [B,T,Hi,Di], dw [B,T,Hi], dk_pooled [B,T//r,Di] and
+    optionally dk_idx [B,T,Di], all fp32.
+    """
+    _need(q, _BF, "q", 4)
+    _need(k, _BF, "k", 4)
+    _need(lse, _F32, "lse", 3)
+    _need(q_idx, _BF, "q_idx", 4)
+    _need(w, _F32, "w", 3)
+    _need(k_pooled, _BF, "k_pooled", 3)
+    _need(kl, _F32, "kl", 2)
+    _need(dq_idx, _F32, "dq_idx", 4)
+    _need(dw, _F32, "dw", 3)
+    _need(dk_pooled, _F32, "dk_pooled", 3)
+    _need(dk_idx, _F32, "dk_idx", 3)
+    _need(ws, torch.uint8, "ws", 1)
+    B, T, Hq, D = q.shape
+    Hkv, Hi, Di = k.shape[2], q_idx.shape[2], q_idx.shape[3]
+    if tuple(k_pooled.shape) != (B, T // r, Di) or tuple(dk_pooled.shape) != (B, T // r, Di):
+        raise ValueError("k_pooled and dk_pooled must be [B, T//r, Di]")
+    scale = D ** -0.5 if scale is None else scale
+    _call("qsa_index_distill", _ptr(q), _ptr(k), _ptr(lse), _ptr(q_idx), _ptr(w),
+          _ptr(k_pooled), B, T, Hq, Hkv, D, Hi, Di, r, scale, _ptr(kl), _ptr(dq_idx), _ptr(dw),
+          _ptr(dk_pooled), _ptr(dk_idx), _ptr(ws), ws.numel(), _stream(stream, q.device))
 
 
 def qsa_check_device_status(ws, stream=None) -> int:

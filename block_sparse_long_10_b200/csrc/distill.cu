@@ -1,0 +1,574 @@
+// Stage-1 indexer distillation: the KL loss between the dense attention's mass
+// on each micro-block and the indexer's softmax over the same blocks, and the
+// gradients of that loss with respect to the indexer's inputs
+// ("用125亿分之6的参数，打平3970亿的旗舰模型", section
+// "稀疏注意力：给检索建索引，也得先学会省纸": the first training stage trains
+// only the indexer, to imitate the full-attention model's distribution, under a
+// KL-divergence loss).
+//
+// Definitions, for query t at position p with candidates j < c = floor(p / 4):
+//   a(t, j)   = sum_h sum_{i<4} exp(scale q_h(t) . k_g(4j + i) - lse_h(t))
+//               (dense causal attention mass of all Hq heads; lse from the main
+//               layer's dense forward)
+//   pi(t, j)  = a(t, j) / Z(t),   Z(t) = sum_{j<c} a(t, j)
+//   s(t, j)   = sum_h w_h(t) max(0, d_h(t, j)),   d_h = q_idx_h(t) . Kp(j)
+//   KL(t)     = sum_j pi (ln pi - s + LSE(t)) = A / Z - ln Z + LSE,
+//               A = sum_j a (ln a - s),  LSE = ln sum_j exp s    (0 when c < 2)
+//   dL/ds     = exp(s - LSE) - pi
+//   dq_idx_h(t) = sum_j dL/ds w_h 1[d_h > 0] Kp(j);   dw_h(t) = sum_j dL/ds max(0, d_h)
+//   dKp(j)    = sum_t sum_h dL/ds w_h 1[d_h > 0] q_idx_h(t);  dk_idx(4j + i) = dKp(j) / 4
+//
+// Three kernels, in stream order:
+//   1. teacher_kernel: the dense Q K^T tiles of the dense prefill kernel
+//      (mma.sync, GQA row packing, cp.async ring) restricted to the candidate
+//      blocks' keys; each probability exp2(S log2e scale - lse log2e) is summed
+//      over the block's 4 keys and the KV group's G heads in registers and
+//      shuffles, and written once per (group, query, block) to the workspace.
+//   2. rows_kernel: one warp per query row; pass 1 over its candidates gives
+//      Z, A and LSE (the row's loss), pass 2 forms dL/ds and accumulates dw
+//      and dq_idx.  Writes (Z, LSE) per row for kernel 3.
+//   3. dkp_kernel: one CTA per 32 blocks; streams the rows that see those
+//      blocks in tiles of 32 (indexer queries staged transposed in shared
+//      memory), recomputes dL/ds and accumulates dKp in registers: a fixed
+//      summation order, no atomics.
+#include "qsa_common.cuh"
+#include "qsa_launch.h"
+
+namespace qsa {
+
+namespace dst {
+
+constexpr int R = 4;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr unsigned FULL = 0xffffffffu;
+
+// ------------------------------------------------------------ teacher --
+constexpr int TW = 8;
+constexpr int TTHREADS = TW * 32;
+constexpr int TROWS = 128;
+constexpr int KT = 64;  // keys per tile (16 blocks)
+constexpr int TSTAGES = 2;
+
+template <int D>
+struct TCfg {
+    static constexpr int ROWB = D * 2;
+    static constexpr int CH = D / 8;
+    static constexpr int TILE = KT * ROWB;
+    static constexpr int BYTES = TSTAGES * TILE;
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(TTHREADS, 2)
+    teacher_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                   const float *__restrict__ lse, int B, int64_t T, int Hkv, int64_t N,
+                   float scale_log2, float *__restrict__ apart, int n_qt) {
+    using C = TCfg<D>;
+    constexpr int TOK = TROWS / G;
+    constexpr int KSTEP = D / 16;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lr = lane >> 2, lc = lane & 3;
+    const int Hq = Hkv * G;
+
+    const int qt = n_qt - 1 - (int)(blockIdx.x % n_qt);  // longest query tiles first
+    const int bg = blockIdx.x / n_qt;
+    const int g = bg % Hkv;
+    const int64_t b = bg / Hkv;
+    const int64_t t0 = (int64_t)qt * TOK;
+
+    // rows lr and lr + 8 of this warp: (token, head) pairs, G heads per token
+    int64_t tok[2], cand[2];
+    int head[2];
+    float lse2[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int r = warp * 16 + lr + e * 8;
+        tok[e] = t0 + r / G;
+        head[e] = g * G + r % G;
+        const bool in = tok[e] < T;
+        cand[e] = in ? tok[e] / R : 0;
+        lse2[e] = in ? lse[(b * T + tok[e]) * Hq + head[e]] * LOG2E : 0.f;
+    }
+    const int64_t t_last = (t0 + TOK - 1 < T) ? t0 + TOK - 1 : T - 1;
+    const int64_t n_keys = (t_last / R) * R;  // keys of the last row's candidate blocks
+    const int n_kt = (int)((n_keys + KT - 1) / KT);
+    if (n_kt == 0) return;
+
+    uint32_t qa[KSTEP][4];
+#pragma unroll
+    for (int ks = 0; ks < KSTEP; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = e & 1, dof = (e >> 1) * 8;
+            uint32_t val = 0;
+            if (tok[rr] < T)
+                val = *reinterpret_cast<const uint32_t *>(
+                    q + ((b * T + tok[rr]) * Hq + head[rr]) * D + ks * 16 + dof + 2 * lc);
+            qa[ks][e] = val;
+        }
+
+    const uint16_t *kbase = k + (b * T) * Hkv * D + g * D;
+    auto load_tile = [&](int kt) {
+        if (kt < n_kt) {
+            uint8_t *dk = smem + (kt % TSTAGES) * C::TILE;
+            for (int i = tid; i < KT * C::CH; i += TTHREADS) {
+                const int kr = i / C::CH, ch = i % C::CH;
+                const int64_t u = (int64_t)kt * KT + kr;
+                const bool ok = u < n_keys;
+                const int64_t off = ok ? u * Hkv * D + ch * 8 : 0;
+                cp_async16(smem_u32(dk + kr * C::ROWB + ((ch ^ (kr & 7)) * 16)), kbase + off,
+                           ok ? 16 : 0);
+            }
+        }
+        cp_async_commit();
+    };
+    load_tile(0);
+
+    float *ag = apart + ((int64_t)g * B + b) * T * N;
+#pragma unroll 1
+    for (int kt = 0; kt < n_kt; ++kt) {
+        cp_async_wait<0>();
+        __syncthreads();
+        load_tile(kt + 1);
+        const uint8_t *sk = smem + (kt % TSTAGES) * C::TILE;
+        float sacc[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KSTEP; ++ks) {
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) {
+                const int mi = lane >> 3;
+                const int kr = pp * 16 + (mi >> 1) * 8 + (lane & 7);
+                const int dc = ks * 2 + (mi & 1);
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(smem_u32(sk + kr * C::ROWB + ((dc ^ (kr & 7)) * 16)), b0, b1, b2, b3);
+                mma_bf16_16816(sacc[2 * pp], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+                mma_bf16_16816(sacc[2 * pp + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2,
+                               b3);
+            }
+        }
+        // Columns nt*8 + 2lc, +1 of this lane belong to block kt*16 + 2nt + (lc >> 1).
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int64_t j = (int64_t)kt * (KT / R) + nt * 2 + (lc >> 1);
+                const bool ok = j < cand[e2];
+                float pr = 0.f;
+                if (ok)
+                    pr = fast_exp2(sacc[nt][e2 * 2] * scale_log2 - lse2[e2]) +
+                         fast_exp2(sacc[nt][e2 * 2 + 1] * scale_log2 - lse2[e2]);
+                pr += __shfl_xor_sync(FULL, pr, 1);  // the block's other two keys
+#pragma unroll
+                for (int off = 4; off < 4 * G; off <<= 1)  // the token's G heads
+                    pr += __shfl_xor_sync(FULL, pr, off);
+                if (ok && (lr % G) == 0 && (lc & 1) == 0) ag[tok[e2] * N + j] = pr;
+            }
+        }
+    }
+    cp_async_wait<0>();
+}
+
+// --------------------------------------------------------------- rows --
+constexpr int RW = 8;  // rows (warps) per CTA
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(RW * 32)
+    rows_kernel(const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
+                const uint16_t *__restrict__ kp, const float *__restrict__ apart, int B,
+                int64_t T, int64_t N, int Hkv, float *__restrict__ kl, float *__restrict__ dq,
+                float *__restrict__ dw, float *__restrict__ dk_idx, float2 *__restrict__ stats,
+                void *status) {
+    constexpr int DPL = DI / 32;  // dims per lane
+    __shared__ __align__(16) float qs_all[RW][HI * DI];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * RW + warp;
+    if (row >= (int64_t)B * T) return;
+    const int64_t b = row / T, t = row % T;
+    const int64_t c = t / R;
+    float *qs = qs_all[warp];
+
+    if (dk_idx && t >= N * R)  // tokens of the trailing partial block: no pooled key
+        for (int kk = lane; kk < DI; kk += 32) dk_idx[row * DI + kk] = 0.f;
+
+    auto zero_row = [&](float Z) {
+        for (int i = lane; i < HI * DI; i += 32) dq[row * HI * DI + i] = 0.f;
+        if (lane < HI) dw[row * HI + lane] = 0.f;
+        if (lane == 0) {
+            kl[row] = 0.f;
+            stats[row] = make_float2(Z, 0.f);
+        }
+    };
+    if (c < 2) {
+        zero_row(1.f);
+        return;
+    }
+
+    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(q_idx + row * HI * DI);
+    for (int i = lane; i < HI * DI / 2; i += 32) {
+        const uint32_t v = qrow[i];
+        qs[2 * i] = bf16_lo(v);
+        qs[2 * i + 1] = bf16_hi(v);
+    }
+    __syncwarp();
+    float wv[HI];
+#pragma unroll
+    for (int h = 0; h < HI; ++h) wv[h] = w[row * HI + h];
+    const uint16_t *kpb = kp + b * N * DI;
+    const float *arow = apart + (b * T + t) * N;
+    const int64_t gstride = (int64_t)B * T * N;
+
+    auto dots = [&](int64_t j, float (&d)[HI]) {
+#pragma unroll
+        for (int h = 0; h < HI; ++h) d[h] = 0.f;
+        const uint4 *kr = reinterpret_cast<const uint4 *>(kpb + j * DI);
+        // not unrolled: the row's queries stay in shared memory (broadcast reads)
+#pragma unroll 1
+        for (int c8 = 0; c8 < DI / 8; ++c8) {
+            const uint4 v = kr[c8];
+            const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+            for (int h = 0; h < HI; ++h) {
+                const float4 qa = *reinterpret_cast<const float4 *>(qs + h * DI + c8 * 8);
+                const float4 qb = *reinterpret_cast<const float4 *>(qs + h * DI + c8 * 8 + 4);
+                d[h] = fmaf(qa.x, x[0], d[h]);
+                d[h] = fmaf(qa.y, x[1], d[h]);
+                d[h] = fmaf(qa.z, x[2], d[h]);
+                d[h] = fmaf(qa.w, x[3], d[h]);
+                d[h] = fmaf(qb.x, x[4], d[h]);
+                d[h] = fmaf(qb.y, x[5], d[h]);
+                d[h] = fmaf(qb.z, x[6], d[h]);
+                d[h] = fmaf(qb.w, x[7], d[h]);
+            }
+        }
+    };
+    auto score = [&](const float (&d)[HI]) {
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < HI; ++h) s = fmaf(wv[h], fmaxf(d[h], 0.f), s);
+        return s;
+    };
+    auto teacher = [&](int64_t j) {
+        float a = 0.f;
+        for (int gg = 0; gg < Hkv; ++gg) a += arow[gg * gstride + j];
+        return a;
+    };
+
+    // pass 1: Z, A and the scores' log-sum-exp
+    float m = -INFINITY, l = 0.f, Z = 0.f, A = 0.f;
+    for (int64_t j = lane; j < c; j += 32) {
+        float d[HI];
+        dots(j, d);
+        const float s = score(d);
+        const float a = teacher(j);
+        if (s > m) {
+            l = l * expf(m - s) + 1.f;
+            m = s;
+        } else {
+            l += expf(s - m);
+        }
+        Z += a;
+        if (a > 0.f) A += a * (logf(a) - s);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+        const float m2 = __shfl_xor_sync(FULL, m, off);
+        const float l2 = __shfl_xor_sync(FULL, l, off);
+        const float mn = fmaxf(m, m2);
+        l = (mn == -INFINITY) ? 0.f : l * expf(m - mn) + l2 * expf(m2 - mn);
+        m = mn;
+        Z += __shfl_xor_sync(FULL, Z, off);
+        A += __shfl_xor_sync(FULL, A, off);
+    }
+    if (!(Z > 0.f)) {  // the teacher's candidate mass vanished in fp32
+        if (lane == 0) record_status(status, QSA_ERR_DEVICE);
+        zero_row(0.f);
+        return;
+    }
+    const float lse_s = m + logf(l);
+    const float inv_z = 1.f / Z;
+
+    // pass 2: dL/ds, then dw and dq_idx
+    float dwa[HI], acc[HI][DPL];
+#pragma unroll
+    for (int h = 0; h < HI; ++h) {
+        dwa[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+    }
+    for (int64_t j0 = 0; j0 < c; j0 += 32) {
+        const int64_t j = j0 + lane;
+        float Gh[HI];
+        if (j < c) {
+            float d[HI];
+            dots(j, d);
+            const float gs = expf(score(d) - lse_s) - teacher(j) * inv_z;
+#pragma unroll
+            for (int h = 0; h < HI; ++h) {
+                dwa[h] = fmaf(gs, fmaxf(d[h], 0.f), dwa[h]);
+                Gh[h] = d[h] > 0.f ? gs * wv[h] : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int h = 0; h < HI; ++h) Gh[h] = 0.f;
+        }
+        const int n = (int)((c - j0) < 32 ? (c - j0) : 32);
+        for (int jj = 0; jj < n; ++jj) {
+            const uint16_t *kr = kpb + (j0 + jj) * DI + lane * DPL;
+            float x[DPL];
+            if constexpr (DPL == 2) {
+                const uint32_t v = *reinterpret_cast<const uint32_t *>(kr);
+                x[0] = bf16_lo(v);
+                x[1] = bf16_hi(v);
+            } else {
+                x[0] = __uint_as_float((uint32_t)kr[0] << 16);
+            }
+#pragma unroll
+            for (int h = 0; h < HI; ++h) {
+                const float gh = __shfl_sync(FULL, Gh[h], jj);
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(gh, x[e], acc[h][e]);
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < HI; ++h) {
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) dq[(row * HI + h) * DI + lane * DPL + e] = acc[h][e];
+        float v = dwa[h];
+#pragma unroll
+        for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
+        if (lane == 0) dw[row * HI + h] = v;
+    }
+    if (lane == 0) {
+        kl[row] = A * inv_z - logf(Z) + lse_s;
+        stats[row] = make_float2(Z, lse_s);
+    }
+}
+
+// ---------------------------------------------------------------- dKp --
+constexpr int JB = 32;  // blocks per CTA
+constexpr int DWARPS = 8;
+constexpr int DTHREADS = DWARPS * 32;
+constexpr int RT = 32;  // rows per tile
+constexpr int BPW = JB / DWARPS;  // blocks per warp
+constexpr int PAD = RT + 1;
+
+template <int HI, int DI>
+struct DCfg {
+    static constexpr int QT = HI * DI * PAD;  // indexer queries, transposed: [h][k][t]
+    static constexpr int KPS = JB * DI;       // pooled keys of the tile
+    static constexpr int AT = JB * PAD;       // teacher mass [j][t]
+    static constexpr int WT = HI * RT;
+    static constexpr int FLOATS = QT + KPS + AT + WT + 2 * RT;
+    static constexpr int BYTES = FLOATS * 4;
+};
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(DTHREADS)
+    dkp_kernel(const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
+               const uint16_t *__restrict__ kp, const float *__restrict__ apart,
+               const float2 *__restrict__ stats, int B, int64_t T, int64_t N, int Hkv, int n_jt,
+               float *__restrict__ dkp, float *__restrict__ dk_idx) {
+    using C = DCfg<HI, DI>;
+    constexpr int DPL = DI / 32;
+    extern __shared__ __align__(16) float sm[];
+    float *qT = sm;
+    float *kpS = qT + C::QT;
+    float *aT = kpS + C::KPS;
+    float *wT = aT + C::AT;
+    float *Zs = wT + C::WT;
+    float *Ls = Zs + RT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int jt = blockIdx.x % n_jt;
+    const int64_t b = blockIdx.x / n_jt;
+    const int64_t j0 = (int64_t)jt * JB;
+    const int nj = (int)((N - j0) < JB ? (N - j0) : JB);
+    const int64_t gstride = (int64_t)B * T * N;
+
+    for (int i = tid; i < C::KPS; i += DTHREADS) {
+        const int jj = i / DI, kk = i % DI;
+        kpS[i] = jj < nj ? __uint_as_float((uint32_t)kp[(b * N + j0 + jj) * DI + kk] << 16)
+                         : 0.f;
+    }
+    float acc[BPW][DPL];
+#pragma unroll
+    for (int q4 = 0; q4 < BPW; ++q4)
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[q4][e] = 0.f;
+
+    // rows that see block j0 as a candidate, and have at least two candidates
+    int64_t t_begin = (j0 + 1) * R;
+    if (t_begin < 2 * R) t_begin = 2 * R;
+    for (int64_t t0 = t_begin; t0 < T; t0 += RT) {
+        __syncthreads();
+        for (int i = tid; i < RT * HI * DI; i += DTHREADS) {
+            const int tt = i / (HI * DI), hk = i % (HI * DI);
+            const int64_t t = t0 + tt;
+            qT[hk * PAD + tt] =
+                t < T ? __uint_as_float((uint32_t)q_idx[(b * T + t) * HI * DI + hk] << 16) : 0.f;
+        }
+        for (int i = tid; i < RT * HI; i += DTHREADS) {
+            const int tt = i / HI, h = i % HI;
+            const int64_t t = t0 + tt;
+            wT[h * RT + tt] = t < T ? w[(b * T + t) * HI + h] : 0.f;
+        }
+        for (int i = tid; i < RT; i += DTHREADS) {
+            const int64_t t = t0 + i;
+            const float2 st = t < T ? stats[b * T + t] : make_float2(0.f, 0.f);
+            Zs[i] = st.x;
+            Ls[i] = st.y;
+        }
+        for (int i = tid; i < RT * JB; i += DTHREADS) {
+            const int tt = i / JB, jj = i % JB;
+            const int64_t t = t0 + tt, j = j0 + jj;
+            float a = 0.f;
+            if (t < T && j < t / R)
+                for (int gg = 0; gg < Hkv; ++gg) a += apart[gg * gstride + (b * T + t) * N + j];
+            aT[jj * PAD + tt] = a;
+        }
+        __syncthreads();
+
+        const int64_t t = t0 + lane;
+        const int64_t ct = t < T ? t / R : 0;
+        const float Zt = Zs[lane], Lt = Ls[lane];
+        const float inv_z = Zt > 0.f ? 1.f / Zt : 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < BPW; ++q4) {
+            const int jl = warp * BPW + q4;
+            if (jl >= nj) break;
+            const int64_t j = j0 + jl;
+            float d[HI];
+#pragma unroll
+            for (int h = 0; h < HI; ++h) d[h] = 0.f;
+#pragma unroll 8
+            for (int kk = 0; kk < DI; ++kk) {
+                const float kv = kpS[jl * DI + kk];
+#pragma unroll
+                for (int h = 0; h < HI; ++h) d[h] = fmaf(qT[(h * DI + kk) * PAD + lane], kv, d[h]);
+            }
+            float s = 0.f;
+#pragma unroll
+            for (int h = 0; h < HI; ++h) s = fmaf(wT[h * RT + lane], fmaxf(d[h], 0.f), s);
+            const bool valid = ct > j && ct >= 2 && Zt > 0.f;
+            const float gs = valid ? expf(s - Lt) - aT[jl * PAD + lane] * inv_z : 0.f;
+            float Gh[HI];
+#pragma unroll
+            for (int h = 0; h < HI; ++h) Gh[h] = d[h] > 0.f ? gs * wT[h * RT + lane] : 0.f;
+#pragma unroll 4
+            for (int tt = 0; tt < RT; ++tt) {
+#pragma unroll
+                for (int h = 0; h < HI; ++h) {
+                    const float gh = __shfl_sync(FULL, Gh[h], tt);
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e)
+                        acc[q4][e] = fmaf(gh, qT[(h * DI + lane * DPL + e) * PAD + tt], acc[q4][e]);
+                }
+            }
+        }
+    }
+
+#pragma unroll
+    for (int q4 = 0; q4 < BPW; ++q4) {
+        const int jl = warp * BPW + q4;
+        if (jl >= nj) break;
+        const int64_t j = j0 + jl;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+            const int kk = lane * DPL + e;
+            dkp[(b * N + j) * DI + kk] = acc[q4][e];
+            if (dk_idx)
+#pragma unroll
+                for (int i = 0; i < R; ++i)
+                    dk_idx[(b * T + j * R + i) * DI + kk] = acc[q4][e] * (1.f / R);
+        }
+    }
+}
+
+template <int D, int G>
+static cudaError_t launch_teacher(const uint16_t *q, const uint16_t *k, const float *lse, int B,
+                                  int64_t T, int Hkv, int64_t N, float scale, float *apart,
+                                  cudaStream_t s) {
+    using C = TCfg<D>;
+    auto kern = teacher_kernel<D, G>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
+    if (e != cudaSuccess) return e;
+    constexpr int TOK = TROWS / G;
+    const int n_qt = (int)((T + TOK - 1) / TOK);
+    const int64_t grid = (int64_t)n_qt * B * Hkv;
+    if (grid == 0) return cudaSuccess;
+    kern<<<(unsigned)grid, TTHREADS, C::BYTES, s>>>(q, k, lse, B, T, Hkv, N, scale * LOG2E, apart,
+                                                   n_qt);
+    return cudaGetLastError();
+}
+
+template <int HI, int DI>
+static cudaError_t launch_indexer_side(const uint16_t *q_idx, const float *w, const uint16_t *kp,
+                                       const float *apart, int B, int64_t T, int64_t N, int Hkv,
+                                       float *kl, float *dq, float *dw, float *dkp, float *dk_idx,
+                                       float2 *stats, void *status, cudaStream_t s) {
+    const int64_t rows = (int64_t)B * T;
+    if (rows > 0) {
+        rows_kernel<HI, DI><<<(unsigned)((rows + RW - 1) / RW), RW * 32, 0, s>>>(
+            q_idx, w, kp, apart, B, T, N, Hkv, kl, dq, dw, dk_idx, stats, status);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (N > 0) {
+        using C = DCfg<HI, DI>;
+        auto kern = dkp_kernel<HI, DI>;
+        cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
+        if (e != cudaSuccess) return e;
+        const int n_jt = (int)((N + JB - 1) / JB);
+        kern<<<(unsigned)((int64_t)n_jt * B), DTHREADS, C::BYTES, s>>>(
+            q_idx, w, kp, apart, stats, B, T, N, Hkv, n_jt, dkp, dk_idx);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
+}
+
+}  // namespace dst
+
+size_t index_distill_ws_bytes(int B, int64_t T, int Hkv) {
+    const int64_t N = T / dst::R;
+    const size_t apart = (size_t)Hkv * B * T * N * sizeof(float);
+    const size_t stats = (size_t)B * T * sizeof(float2);
+    return kWsHeader + ((apart + 15) & ~(size_t)15) + stats;
+}
+
+cudaError_t launch_index_distill(const uint16_t *q, const uint16_t *k, const float *lse,
+                                 const uint16_t *q_idx, const float *w, const uint16_t *kp, int B,
+                                 int64_t T, int Hq, int Hkv, int D, int Hi, int Di, float scale,
+                                 float *kl, float *dq, float *dw, float *dkp, float *dk_idx,
+                                 void *ws, cudaStream_t s) {
+    const int64_t N = T / dst::R;
+    const size_t apart_bytes = (size_t)Hkv * B * T * N * sizeof(float);
+    float *apart = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kWsHeader);
+    float2 *stats = reinterpret_cast<float2 *>(static_cast<uint8_t *>(ws) + kWsHeader +
+                                               ((apart_bytes + 15) & ~(size_t)15));
+    const int G = Hq / Hkv;
+    cudaError_t e = cudaErrorInvalidValue;
+    if (N > 0) {
+#define QSA_TEACHER(D_, G_) \
+    if (D == D_ && G == G_) e = dst::launch_teacher<D_, G_>(q, k, lse, B, T, Hkv, N, scale, apart, s);
+        QSA_TEACHER(64, 1) QSA_TEACHER(64, 2) QSA_TEACHER(64, 4) QSA_TEACHER(64, 8)
+        QSA_TEACHER(128, 1) QSA_TEACHER(128, 2) QSA_TEACHER(128, 4) QSA_TEACHER(128, 8)
+#undef QSA_TEACHER
+        if (e != cudaSuccess) return e;
+    }
+    e = cudaErrorInvalidValue;
+#define QSA_IDX_SIDE(HI_, DI_)                                                                   \
+    if (Hi == HI_ && Di == DI_)                                                                  \
+        e = dst::launch_indexer_side<HI_, DI_>(q_idx, w, kp, apart, B, T, N, Hkv, kl, dq, dw, dkp, \
+                                               dk_idx, stats, ws, s);
+    QSA_IDX_SIDE(1, 32) QSA_IDX_SIDE(2, 32) QSA_IDX_SIDE(4, 32)
+    QSA_IDX_SIDE(1, 64) QSA_IDX_SIDE(2, 64) QSA_IDX_SIDE(4, 64)
+#undef QSA_IDX_SIDE
+    return e;
+}
+
+}  // namespace qsa

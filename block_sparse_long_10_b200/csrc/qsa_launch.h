@@ -67,6 +67,15 @@ cudaError_t launch_split_decode(const uint16_t *q, const uint16_t *k, const uint
                                 float scale, uint16_t *o, float *lse, float *part,
                                 void *status, int num_sms, cudaStream_t s);
 
+// Stage-1 indexer distillation (distill.cu); the workspace holds the teacher's
+// block mass per KV group and the per-row (Z, LSE) after the 256-byte header.
+size_t index_distill_ws_bytes(int B, int64_t T, int Hkv);
+cudaError_t launch_index_distill(const uint16_t *q, const uint16_t *k, const float *lse,
+                                 const uint16_t *q_idx, const float *w, const uint16_t *kp, int B,
+                                 int64_t T, int Hq, int Hkv, int D, int Hi, int Di, float scale,
+                                 float *kl, float *dq, float *dw, float *dkp, float *dk_idx,
+                                 void *ws, cudaStream_t s);
+
 cudaError_t launch_dense_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
                                  int64_t T, int Hq, int Hkv, int D, float scale, uint16_t *o,
                                  float *lse, cudaStream_t s);

@@ -234,6 +234,50 @@ QSA_API qsa_status_t qsa_dense_gqa_decode(const qsa_bf16_t *q, const qsa_bf16_t 
                                   size_t ws_bytes, void *stream);
 
 /*
+ * Stage-1 indexer distillation: loss and indexer gradients [ART: QSA is trained
+ * in two stages; the first, dense distillation, trains only the indexer, to
+ * imitate the full-attention model's attention distribution, with a
+ * KL-divergence loss; SUM: QSA first distils the dense attention distribution].
+ *
+ * For query t of batch row b at position p = t, with candidates the complete
+ * blocks j < c = floor(p / r) (the blocks qsa_index_topk ranks):
+ *   a(t, j)  = sum over all Hq heads h and the r tokens u of block j of
+ *              exp(scale * q[b,t,h] . k[b,u,h/(Hq/Hkv)] - lse[b,t,h])
+ *   pi(t, j) = a(t, j) / sum_{j' < c} a(t, j')          (the teacher)
+ *   s(t, j)  = sum_h w[b,t,h] * max(0, q_idx[b,t,h,:] . k_pooled[b,j,:])
+ *   kl[b,t]  = KL(pi(t, .) || softmax_j s(t, .)), 0 when c < 2
+ * and the gradients of L = sum_{b,t} kl[b,t] (the teacher is a constant), with
+ * g(t, j) = softmax_j s(t, j) - pi(t, j) and the ReLU's derivative 1[x > 0]:
+ *   dq_idx[b,t,h,:] = sum_j g w_h 1[q_idx_h . Kp_j > 0] k_pooled[b,j,:]
+ *   dw[b,t,h]       = sum_j g max(0, q_idx_h . Kp_j)
+ *   dk_pooled[b,j,:] = sum_t sum_h g w_h 1[q_idx_h . Kp_j > 0] q_idx[b,t,h,:]
+ *   dk_idx[b,u,:]   = dk_pooled[b, u / r, :] / r for u < r * floor(T / r), else 0
+ *                     (the bf16 rounding of the pooled key taken as identity)
+ *   q, k     [B, T, Hq, D] / [B, T, Hkv, D] bf16: the main attention's inputs
+ *   lse      [B, T, Hq] fp32: natural-log softmax normalisers of the dense
+ *            causal attention at `scale` (qsa_dense_gqa_prefill writes them)
+ *   q_idx [B, T, Hi, Di] bf16, w [B, T, Hi] fp32, k_pooled [B, floor(T/r), Di]
+ *            bf16 (qsa_pool of the indexer keys; NULL allowed when T < r)
+ *   kl [B, T], dq_idx [B, T, Hi, Di], dw [B, T, Hi], dk_pooled [B, floor(T/r), Di]
+ *            fp32 outputs; dk_idx [B, T, Di] fp32 or NULL
+ *   ws       at least qsa_index_distill_workspace_size(B, T, Hkv, r) bytes,
+ *            first 256 bytes zeroed once (status word); it holds the teacher's
+ *            block mass, 4 * Hkv * B * T * floor(T / r) bytes (about Hkv * B * T^2)
+ * A row whose teacher mass on every candidate underflows fp32 gets zero loss and
+ * gradients and records QSA_ERR_DEVICE.  T == 0 is a no-op.  Constraints: r = 4,
+ * the attention shapes of qsa_dense_gqa_prefill, the indexer shapes of
+ * qsa_index_topk.
+ */
+QSA_API size_t qsa_index_distill_workspace_size(int B, int64_t T, int Hkv, int r);
+QSA_API qsa_status_t qsa_index_distill(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                       const float *lse, const qsa_bf16_t *q_idx,
+                                       const float *w, const qsa_bf16_t *k_pooled, int B,
+                                       int64_t T, int Hq, int Hkv, int D, int Hi, int Di,
+                                       int r, float scale, float *kl, float *dq_idx, float *dw,
+                                       float *dk_pooled, float *dk_idx, void *ws,
+                                       size_t ws_bytes, void *stream);
+
+/*
  * Synchronises `stream`, reads the status word kernels recorded at the start
  * of `ws`, clears it, and returns it (QSA_OK if nothing was recorded).  The
  * word is sticky: it keeps the first error recorded by any call that used

@@ -124,6 +124,29 @@ def test_attention_validation(lib):
                                     f, None, f, m - 1, s) == WORKSPACE
 
 
+def test_index_distill_validation(lib):
+    f, s = _fake(), _nullp()
+    n = lib.qsa_index_distill_workspace_size(1, 2048, 1, 4)
+    assert n == 256 + 2048 * 512 * 4 + 2048 * 8
+    assert lib.qsa_index_distill_workspace_size(1, 2048, 1, 2) == SIZE_MAX
+    assert lib.qsa_index_distill_workspace_size(0, 2048, 1, 4) == SIZE_MAX
+    base = dict(q=f, k=f, lse=f, qi=f, w=f, kp=f, B=1, T=2048, Hq=4, Hkv=1, D=64, Hi=2, Di=32,
+                r=4, scale=ctypes.c_float(0.125), kl=f, dq=f, dw=f, dkp=f, dki=None, ws=f, wsb=n)
+    call = lambda **kw: lib.qsa_index_distill(*dict(base, **kw).values(), s)
+    assert call(Hq=5, Hkv=2) == INVALID                  # Hq % Hkv
+    assert call(lse=_nullp()) == INVALID
+    assert call(dkp=_nullp()) == INVALID                 # needed when T >= r
+    assert call(scale=ctypes.c_float(float("nan"))) == INVALID
+    assert call(r=8) == UNSUPPORTED
+    assert call(D=96) == UNSUPPORTED
+    assert call(Hi=3) == UNSUPPORTED
+    assert call(Hq=16, Hkv=1) == UNSUPPORTED             # G = 16
+    assert call(wsb=n - 1) == WORKSPACE
+    assert call(ws=_nullp()) == WORKSPACE
+    assert call(q=_fake(0x10008)) == INVALID              # misaligned
+    assert call(T=0) == OK
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(qsa, "_LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(qsa, "_lib", None)
