@@ -461,6 +461,51 @@ def extra_decode(qsa, device, peaks, flush):
     return out
 
 
+def extra_distill(qsa, device, peaks, flush):
+    """Stage-1 indexer distillation (qsa_index_distill) at 32K tokens: the dense
+    forward's lse and the pooled keys are made once, outside the timed call."""
+    w = synth.WORKLOADS["prefill-32k"]
+    x = synth.make_prefill(w, device)
+    B, T, N = w.B, w.T, w.T // w.r
+    f32 = dict(dtype=torch.float32, device=device)
+    o = torch.empty_like(x["q"])
+    lse = torch.empty(B, T, w.Hq, **f32)
+    qsa.qsa_dense_gqa_prefill(x["q"], x["k"], x["v"], o, w.scale, lse=lse)
+    kp = torch.empty(B, N, w.Di, dtype=BF, device=device)
+    qsa.qsa_pool(x["k_idx"], kp, w.r)
+    kl = torch.empty(B, T, **f32)
+    dq = torch.empty(B, T, w.Hi, w.Di, **f32)
+    dw = torch.empty(B, T, w.Hi, **f32)
+    dkp = torch.empty(B, N, w.Di, **f32)
+    dki = torch.empty(B, T, w.Di, **f32)
+    ws = qsa.workspace(qsa.qsa_index_distill_workspace_size(B, T, w.Hkv, w.r), device)
+    s = torch.cuda.current_stream(device)
+    call = lambda: qsa.qsa_index_distill(x["q"], x["k"], lse, x["q_idx"], x["w"], kp, kl, dq,
+                                         dw, dkp, ws, w.r, w.scale, dk_idx=dki, stream=s)
+    ms = time_call(call, s, 3, 1, flush)
+    status = qsa.qsa_check_device_status(ws)
+    # teacher: 2 Hq D FLOP per (query, key) pair over the candidate blocks' keys
+    teacher_flops = 2.0 * w.Hq * w.D * sum_candidate_keys(T, w.r)
+    pairs = sum_candidate_keys(T, w.r) / w.r
+    out = {"workload": w.name, "ms": ms, "status": status,
+           "teacher_flops": teacher_flops,
+           "teacher_tflops_if_whole_call": teacher_flops / (ms / 1e3) / 1e12,
+           "row_block_pairs": pairs, "kl_mean": float(kl.mean()),
+           "finite": bool(torch.isfinite(dq).all() and torch.isfinite(dkp).all()),
+           "l2": "flushed between iterations"}
+    del x, o, lse, kp, kl, dq, dw, dkp, dki, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def sum_candidate_keys(T: int, r: int) -> float:
+    """Sum over query rows p < T of r * floor(p / r): the keys of every row's
+    candidate blocks (exact integer arithmetic)."""
+    m, rem = divmod(T, r)           # rows p = r*c + i: m full groups, then rem rows of c = m
+    full = r * r * (m * (m - 1) // 2)  # sum over c < m of r rows x r*c keys
+    return float(full + rem * r * m)
+
+
 # ------------------------------------------------------------ CPU oracle --
 
 def oracle_sample(w: synth.Workload, x: dict, n_rows: int, seed: int, threads: int | None = None):
@@ -547,7 +592,7 @@ def main():
     ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
     ap.add_argument("--workload", default="prefill-1m",
                     choices=[n for n, w in synth.WORKLOADS.items() if w.kind == "prefill"])
-    ap.add_argument("--no-extra", action="store_true", help="skip 128K and decode lines")
+    ap.add_argument("--no-extra", action="store_true", help="skip the 128K, decode and distillation lines")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense GQA ratio run")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -636,6 +681,10 @@ def main():
             if w.name != "prefill-128k":
                 line["extra"]["prefill-128k"] = extra_prefill(qsa, "prefill-128k", device, peaks, fl)
             line["extra"]["decode-256k-b64"] = extra_decode(qsa, device, peaks, fl)
+            try:  # a secondary measurement: report a failure instead of losing the line
+                line["extra"]["distill-32k"] = extra_distill(qsa, device, peaks, fl)
+            except Exception as exc:
+                line["extra"]["distill-32k"] = {"error": f"{type(exc).__name__}: {exc}"}
         print(json.dumps(line), flush=True)
     barrier(world)
     if world > 1:
