@@ -484,12 +484,18 @@ def extra_distill(qsa, device, peaks, flush):
                                          dw, dkp, ws, w.r, w.scale, dk_idx=dki, stream=s)
     ms = time_call(call, s, 3, 1, flush)
     status = qsa.qsa_check_device_status(ws)
-    # teacher: 2 Hq D FLOP per (query, key) pair over the candidate blocks' keys
+    # teacher: 2 Hq D FLOP per (query, key) pair over the candidate blocks' keys;
+    # indexer side: per (row, block) pair the scores (2 Hi Di), and the dq_idx and
+    # dKp products (2 Hi Di each)
     teacher_flops = 2.0 * w.Hq * w.D * sum_candidate_keys(T, w.r)
     pairs = sum_candidate_keys(T, w.r) / w.r
+    flops = teacher_flops + pairs * 3 * 2 * w.Hi * w.Di
+    achieved = flops / (ms / 1e3) / 1e12
     out = {"workload": w.name, "ms": ms, "status": status,
            "teacher_flops": teacher_flops,
            "teacher_tflops_if_whole_call": teacher_flops / (ms / 1e3) / 1e12,
+           "roofline": dict(roof(achieved, peaks["bf16_tflops"], "TFLOP/s", "tensor"),
+                            scope="whole call, algorithmic FLOPs (teacher + indexer side)"),
            "row_block_pairs": pairs, "kl_mean": float(kl.mean()),
            "finite": bool(torch.isfinite(dq).all() and torch.isfinite(dkp).all()),
            "l2": "flushed between iterations"}
