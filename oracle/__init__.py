@@ -9,6 +9,11 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  It never imports the CUDA library and the CUDA
 library never imports it.
 
+Submodules (numpy, fp64), each stating its readings of the pages:
+``distill`` (stage-1 indexer distillation: KL loss and indexer gradients),
+``sparse_train`` (stage-2: sparse attention backward, indexer loss over the
+selection) and ``gdn`` (the gated delta rule of the hybrid's GDN layers).
+
 Sources are cited in ``qsa_oracle.c``'s header: the article
 "用125亿分之6的参数，打平3970亿的旗舰模型" (section "稀疏注意力：给检索建索引，也得先学会省纸"),
 the paper summary "On the Design of Qwen3.8-Next Architecture" (token-mixing
