@@ -27,7 +27,8 @@ __all__ = [
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode_noalloc",
     "qsa_dense_gqa_prefill",
     "qsa_dense_gqa_decode", "qsa_dense_gqa_decode_workspace_size",
-    "qsa_index_distill", "qsa_index_distill_workspace_size",
+    "qsa_index_distill", "qsa_index_distill_workspace_size", "qsa_sparse_attn_backward",
+    "qsa_gdn_prefill", "qsa_gdn_decode",
     "qsa_check_device_status", "qsa_status_string", "qsa_version",
 ]
 
@@ -74,6 +75,11 @@ _SIGS = {
     "qsa_dense_gqa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "qsa_dense_gqa_decode": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _F,
                                   _VP, _VP, _VP, _SZ, _VP]),
+    "qsa_sparse_attn_backward": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
+                                      _F, _VP, _VP, _VP, _VP]),
+    "qsa_gdn_prefill": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP,
+                             _VP]),
+    "qsa_gdn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP, _VP]),
     "qsa_index_distill_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "qsa_index_distill": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
                                _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -293,6 +299,57 @@ def qsa_dense_gqa_decode(q, k_cache, v_cache, seqlens, o, ws, scale=None, lse=No
     scale = D ** -0.5 if scale is None else scale
     _call("qsa_dense_gqa_decode", _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), L, B,
           Hq, Hkv, D, scale, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream, q.device))
+
+
+# ------------------------------------------------ sparse attention backward --
+
+def qsa_sparse_attn_backward(q, k, v, sel, d_o, dq, dk, dv, r=4, budget=2048, scale=None,
+                             stream=None):
+    """Gradients of the sparse prefill attention for an output gradient d_o:
+    q, d_o [B,T,Hq,D], k/v [B,T,Hkv,D] bf16, sel [B,T,kb] -> dq [B,T,Hq,D],
+    dk/dv [B,T,Hkv,D] fp32 (overwritten)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
+        _need(t, _BF, n, 4)
+    _need(sel, _I32, "sel", 3)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, _F32, n, 4)
+    B, T, Hq, D = q.shape
+    scale = D ** -0.5 if scale is None else scale
+    _call("qsa_sparse_attn_backward", _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(d_o), B, T,
+          Hq, k.shape[2], D, r, budget, scale, _ptr(dq), _ptr(dk), _ptr(dv),
+          _stream(stream, q.device))
+
+
+# ------------------------------------------------------------ Gated DeltaNet --
+
+def qsa_gdn_prefill(q, k, v, alpha, beta, o, state_out, state_in=None, stream=None):
+    """Gated delta rule over a prefill: q, k [B,T,H,dk], v [B,T,H,dv] bf16,
+    alpha, beta [B,T,H] fp32, state_in [B,H,dv,dk] fp32 or None ->
+    o [B,T,H,dv] fp32, state_out [B,H,dv,dk] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, _BF, n, 4)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _need(t, _F32, n, 3)
+    _need(o, _F32, "o", 4)
+    _need(state_out, _F32, "state_out", 4)
+    _need(state_in, _F32, "state_in", 4)
+    B, T, H, dk = k.shape
+    _call("qsa_gdn_prefill", _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in),
+          B, T, H, dk, v.shape[3], _ptr(o), _ptr(state_out), _stream(stream, k.device))
+
+
+def qsa_gdn_decode(q, k, v, alpha, beta, state, o, stream=None):
+    """One token per sequence: q, k [B,H,dk], v [B,H,dv] bf16, alpha, beta [B,H]
+    fp32; state [B,H,dv,dk] fp32 updated in place; o [B,H,dv] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, _BF, n, 3)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _need(t, _F32, n, 2)
+    _need(state, _F32, "state", 4)
+    _need(o, _F32, "o", 3)
+    B, H, dk = k.shape
+    _call("qsa_gdn_decode", _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), B,
+          H, dk, v.shape[2], _ptr(o), _stream(stream, k.device))
 
 
 # ----------------------------------------------------- indexer distillation --

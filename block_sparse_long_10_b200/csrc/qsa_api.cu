@@ -294,6 +294,65 @@ qsa_status_t qsa_dense_gqa_decode(const qsa_bf16_t *q, const qsa_bf16_t *k_cache
                                               ws, sms, static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------- sparse attention backward --
+qsa_status_t qsa_sparse_attn_backward(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                      const qsa_bf16_t *v, const int32_t *sel,
+                                      const qsa_bf16_t *d_o, int B, int64_t T, int Hq, int Hkv,
+                                      int D, int r, int budget, float scale, float *dq,
+                                      float *dk, float *dv, void *stream) {
+    if (B < 1 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || D < 1 || r < 1 ||
+        budget < r || budget % r != 0 || !(scale == scale))
+        return QSA_ERR_INVALID_ARG;
+    if (T == 0) return QSA_OK;
+    if (!q || !k || !v || !sel || !d_o || !dq || !dk || !dv) return QSA_ERR_INVALID_ARG;
+    const int kb = budget / r;
+    if (r != 4 || !supported_attn(Hq, Hkv, D) || kb > 1024) return QSA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv))
+        return QSA_ERR_INVALID_ARG;
+    int sms = 0;
+    qsa_status_t st = current_device(&sms);
+    if (st != QSA_OK) return st;
+    return from_cuda(qsa::launch_sparse_attn_backward(q, k, v, sel, d_o, B, T, Hq, Hkv, D, kb,
+                                                      scale, dq, dk, dv,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------- Gated DeltaNet --
+static bool supported_gdn(int dk, int dv) {
+    return (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
+}
+
+qsa_status_t qsa_gdn_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k, const qsa_bf16_t *v,
+                             const float *alpha, const float *beta, const float *state_in, int B,
+                             int64_t T, int H, int dk, int dv, float *o, float *state_out,
+                             void *stream) {
+    if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return QSA_ERR_INVALID_ARG;
+    if (!state_out || (T > 0 && (!q || !k || !v || !alpha || !beta || !o)))
+        return QSA_ERR_INVALID_ARG;
+    if (!supported_gdn(dk, dv)) return QSA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(state_out) || (state_in && !aligned16(state_in))) return QSA_ERR_INVALID_ARG;
+    int sms = 0;
+    qsa_status_t st = current_device(&sms);
+    if (st != QSA_OK) return st;
+    return from_cuda(qsa::launch_gdn_prefill(q, k, v, alpha, beta, state_in, B, T, H, dk, dv, o,
+                                             state_out, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status_t qsa_gdn_decode(const qsa_bf16_t *q, const qsa_bf16_t *k, const qsa_bf16_t *v,
+                            const float *alpha, const float *beta, float *state, int B, int H,
+                            int dk, int dv, float *o, void *stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return QSA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !alpha || !beta || !state || !o) return QSA_ERR_INVALID_ARG;
+    if (!supported_gdn(dk, dv)) return QSA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(state)) return QSA_ERR_INVALID_ARG;
+    int sms = 0;
+    qsa_status_t st = current_device(&sms);
+    if (st != QSA_OK) return st;
+    return from_cuda(qsa::launch_gdn_decode(q, k, v, alpha, beta, state, B, H, dk, dv, o,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------- indexer distillation --
 size_t qsa_index_distill_workspace_size(int B, int64_t T, int Hkv, int r) {
     if (B < 1 || T < 0 || Hkv < 1 || r != 4) return SIZE_MAX;

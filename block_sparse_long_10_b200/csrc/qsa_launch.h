@@ -76,6 +76,21 @@ cudaError_t launch_index_distill(const uint16_t *q, const uint16_t *k, const flo
                                  float *kl, float *dq, float *dw, float *dkp, float *dk_idx,
                                  void *ws, cudaStream_t s);
 
+// Backward of the sparse prefill attention (sparse_bwd.cu); zeroes dk and dv first.
+cudaError_t launch_sparse_attn_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                        const int32_t *sel, const uint16_t *dout, int B,
+                                        int64_t T, int Hq, int Hkv, int D, int kb, float scale,
+                                        float *dq, float *dk, float *dv, cudaStream_t s);
+
+// Gated delta rule (gdn.cu): exact recurrence, one CTA per (sequence, head).
+cudaError_t launch_gdn_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                               const float *alpha, const float *beta, const float *state_in,
+                               int B, int64_t T, int H, int dk, int dv, float *o,
+                               float *state_out, cudaStream_t s);
+cudaError_t launch_gdn_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              const float *alpha, const float *beta, float *state, int B, int H,
+                              int dk, int dv, float *o, cudaStream_t s);
+
 cudaError_t launch_dense_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
                                  int64_t T, int Hq, int Hkv, int D, float scale, uint16_t *o,
                                  float *lse, cudaStream_t s);

@@ -234,6 +234,31 @@ QSA_API qsa_status_t qsa_dense_gqa_decode(const qsa_bf16_t *q, const qsa_bf16_t 
                                   size_t ws_bytes, void *stream);
 
 /*
+ * Backward of the sparse prefill attention, for the second training stage
+ * [ART: after the dense distillation, the indexer and the backbone are trained
+ * together on the sparse pattern].  The selection is held fixed.  With the
+ * forward of qsa_sparse_attn_prefill (q_pos0 NULL: query t at p = t, token set
+ * S(t) = { r*j + i <= p : j in sel[b, t, :], j >= 0 }, P the softmax of
+ * scale * q . k over S(t)) and an output gradient d_o:
+ *   D_h      = sum_{u in S} P(u) (d_o_h . v_g(u))
+ *   dS(u)    = P(u) (d_o_h . v_g(u) - D_h)
+ *   dq_h     = scale * sum_{u in S} dS(u) k_g(u)
+ *   dk_g(u) += scale * dS(u) q_h;   dv_g(u) += P(u) d_o_h
+ * summed over every query and head that reads token u (g = h / (Hq / Hkv)).
+ *   q, d_o [B, T, Hq, D] bf16; k, v [B, T, Hkv, D] bf16; sel [B, T, budget/r]
+ *   int32 (distinct entries; negative or future blocks ignored);
+ *   dq [B, T, Hq, D], dk, dv [B, T, Hkv, D] fp32 outputs (overwritten).
+ * Softmax statistics are recomputed (no forward lse needed); dk and dv are
+ * accumulated with atomics, so their low-order bits vary from run to run.
+ * T == 0 is a no-op.  Shapes as for qsa_sparse_attn_prefill.
+ */
+QSA_API qsa_status_t qsa_sparse_attn_backward(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                              const qsa_bf16_t *v, const int32_t *sel,
+                                              const qsa_bf16_t *d_o, int B, int64_t T, int Hq,
+                                              int Hkv, int D, int r, int budget, float scale,
+                                              float *dq, float *dk, float *dv, void *stream);
+
+/*
  * Stage-1 indexer distillation: loss and indexer gradients [ART: QSA is trained
  * in two stages; the first, dense distillation, trains only the indexer, to
  * imitate the full-attention model's attention distribution, with a
@@ -276,6 +301,30 @@ QSA_API qsa_status_t qsa_index_distill(const qsa_bf16_t *q, const qsa_bf16_t *k,
                                        int r, float scale, float *kl, float *dq_idx, float *dw,
                                        float *dk_pooled, float *dk_idx, void *ws,
                                        size_t ws_bytes, void *stream);
+
+/*
+ * Gated DeltaNet token mixing, the hybrid's other layers [ART: GDN keeps a
+ * matrix state and, for each token, writes the error between the token's
+ * information and what the memory holds for it, under a decay gate and a write
+ * gate; SUM: a fixed-size recurrent state with a decay gate and delta writes].
+ * Per (sequence b, head h), state S in R^{dv x dk} (fp32), per token t:
+ *   S_t = alpha_t S_{t-1} + beta_t (v_t - alpha_t S_{t-1} k_t) k_t^T,   o_t = S_t q_t
+ * (keys, queries and gates as given: normalisation and scaling are the caller's).
+ *   q, k [B, T, H, dk] bf16; v [B, T, H, dv] bf16; alpha, beta [B, T, H] fp32;
+ *   state_in [B, H, dv, dk] fp32 or NULL (zeros); o [B, T, H, dv] fp32;
+ *   state_out [B, H, dv, dk] fp32 (may be state_in).  dk, dv in {64, 128}.
+ * T == 0 copies the initial state.  Decode is one token per sequence with the
+ * state updated in place: q, k [B, H, dk], v [B, H, dv], alpha, beta [B, H],
+ * state [B, H, dv, dk], o [B, H, dv].
+ */
+QSA_API qsa_status_t qsa_gdn_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                     const qsa_bf16_t *v, const float *alpha, const float *beta,
+                                     const float *state_in, int B, int64_t T, int H, int dk,
+                                     int dv, float *o, float *state_out, void *stream);
+QSA_API qsa_status_t qsa_gdn_decode(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                    const qsa_bf16_t *v, const float *alpha, const float *beta,
+                                    float *state, int B, int H, int dk, int dv, float *o,
+                                    void *stream);
 
 /*
  * Synchronises `stream`, reads the status word kernels recorded at the start

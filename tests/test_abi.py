@@ -147,6 +147,38 @@ def test_index_distill_validation(lib):
     assert call(T=0) == OK
 
 
+def test_sparse_attn_backward_validation(lib):
+    f, s = _fake(), _nullp()
+    base = dict(q=f, k=f, v=f, sel=f, do=f, B=1, T=64, Hq=16, Hkv=2, D=128, r=4, budget=2048,
+                scale=ctypes.c_float(0.1), dq=f, dk=f, dv=f)
+    call = lambda **kw: lib.qsa_sparse_attn_backward(*dict(base, **kw).values(), s)
+    assert call(Hq=15) == INVALID
+    assert call(budget=2047) == INVALID
+    assert call(do=_nullp()) == INVALID
+    assert call(dk=_fake(0x10004)) == INVALID               # misaligned
+    assert call(D=96) == UNSUPPORTED
+    assert call(r=2, budget=2048) == UNSUPPORTED
+    assert call(budget=8192) == UNSUPPORTED                 # kb > 1024
+    assert call(T=0) == OK
+
+
+def test_gdn_validation(lib):
+    f, s = _fake(), _nullp()
+    pre = lambda **kw: lib.qsa_gdn_prefill(*dict(dict(
+        q=f, k=f, v=f, a=f, b=f, s0=None, B=1, T=64, H=4, dk=128, dv=128, o=f, s1=f),
+        **kw).values(), s)
+    assert pre(H=0) == INVALID
+    assert pre(s1=_nullp()) == INVALID
+    assert pre(a=_nullp()) == INVALID
+    assert pre(dk=96) == UNSUPPORTED
+    assert pre(s1=_fake(0x10008)) == INVALID                 # misaligned state
+    dec = lambda **kw: lib.qsa_gdn_decode(*dict(dict(
+        q=f, k=f, v=f, a=f, b=f, st=f, B=2, H=4, dk=64, dv=64, o=f), **kw).values(), s)
+    assert dec(B=0) == INVALID
+    assert dec(st=_nullp()) == INVALID
+    assert dec(dv=32) == UNSUPPORTED
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(qsa, "_LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(qsa, "_lib", None)
