@@ -23,7 +23,7 @@ from block_sparse_long_10_b200 import synth
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 BF = torch.bfloat16
-W_SMALL = synth.Workload("cp-small", "prefill", 1, 256, 4, 2, 64, 2, 32, 4, 64, 5, 4)
+W_SMALL = synth.Workload("cp-small", "prefill", 1, 240, 4, 2, 64, 2, 32, 4, 64, 5, 4)  # 2·W·r | 240 for W = 1, 2, 3
 
 
 def _free_port():
@@ -174,20 +174,22 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_context_parallel_equals_one_shot_oracle_gloo():
+@pytest.mark.parametrize("world", [2, 3])
+def test_multi_rank_context_parallel_equals_one_shot_oracle_gloo(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(300)
         assert p.exitcode == 0
-    res = dict(q.get(timeout=10) for _ in range(2))
-    assert res[1] == {"k_round_trip": True, "pooled_in_place": True}
-    assert res[0] == {"k_round_trip": True, "pooled_in_place": True, "sel": True, "o": True, "lse": True,
-                      "needles": True}
+    res = dict(q.get(timeout=10) for _ in range(world))
+    for r in range(1, world):
+        assert res[r] == {"k_round_trip": True, "pooled_in_place": True}
+    assert res[0] == {"k_round_trip": True, "pooled_in_place": True, "sel": True, "o": True,
+                      "lse": True, "needles": True}
 
 
 # ------------------------------------------------------------------- GPU --
