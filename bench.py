@@ -484,6 +484,7 @@ def extra_distill(qsa, device, peaks, flush):
                                          dw, dkp, ws, w.r, w.scale, dk_idx=dki, stream=s)
     ms = time_call(call, s, 3, 1, flush)
     status = qsa.qsa_check_device_status(ws)
+    cpu = distill_oracle_sample(w, x, 16, seed=7)
     # teacher: 2 Hq D FLOP per (query, key) pair over the candidate blocks' keys;
     # indexer side: per (row, block) pair the scores (2 Hi Di), and the dq_idx and
     # dKp products (2 Hi Di each)
@@ -497,11 +498,36 @@ def extra_distill(qsa, device, peaks, flush):
            "roofline": dict(roof(achieved, peaks["bf16_tflops"], "TFLOP/s", "tensor"),
                             scope="whole call, algorithmic FLOPs (teacher + indexer side)"),
            "row_block_pairs": pairs, "kl_mean": float(kl.mean()),
+           "cpu_baseline": cpu,
            "finite": bool(torch.isfinite(dq).all() and torch.isfinite(dkp).all()),
            "l2": "flushed between iterations"}
     del x, o, lse, kp, kl, dq, dw, dkp, dki, ws
     torch.cuda.empty_cache()
     return out
+
+
+def distill_oracle_sample(w: synth.Workload, x: dict, n_rows: int, seed: int) -> dict:
+    """The distillation oracle (numpy, fp64) on stratified rows of the workload;
+    the mean time per row, times T, estimates one whole call."""
+    from oracle import distill  # test/baseline infrastructure only
+    import oracle
+    host = {n: oracle.bf16_bits_to_f64(synth.bf16_bits(x[n])[0])
+            for n in ("q", "k", "q_idx", "k_idx")}
+    kp = oracle.bf16_bits_to_f64(oracle.pool(synth.bf16_bits(x["k_idx"]), w.r)[0])
+    wt = x["w"][0].cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(seed)
+    edges = np.linspace(0, w.T, n_rows + 1).astype(np.int64)
+    rows = np.array([rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))
+                     for i in range(n_rows)], np.int64)
+    t0 = time.perf_counter()
+    distill.distill_rows_f64(host["q"], host["k"], host["q_idx"], wt, kp, w.r, w.scale,
+                             rows=rows)
+    secs = time.perf_counter() - t0
+    est_ms = secs / n_rows * w.T * 1e3
+    return {"value": est_ms, "unit": "ms per call (extrapolated)", "cores": cpu_cores(),
+            "kind": "oracle",
+            "sample": f"{n_rows} stratified query rows of {w.name}, {secs:.1f} s wall; mean "
+                      f"time per row times {w.T} rows"}
 
 
 def sum_candidate_keys(T: int, r: int) -> float:
