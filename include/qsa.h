@@ -3,7 +3,10 @@
  * Sparse Attention (QSA) layer: micro-block pooling, a lightweight MQA
  * indexer with top-k block selection, and exact softmax attention over the
  * tokens of the selected blocks, for prefill and decode; plus dense causal
- * GQA attention on the same tensors (the speed-up baseline).
+ * GQA attention on the same tensors (the speed-up baseline).  For training,
+ * the first stage's indexer distillation loss and gradients and the second
+ * stage's sparse attention backward; and the gated delta rule of the
+ * hybrid's Gated DeltaNet layers (prefill and decode).
  *
  * Sources (web pages about the Qwen3.8-Flash-Next architecture):
  *   [ART]  "用125亿分之6的参数，打平3970亿的旗舰模型", section
