@@ -699,12 +699,19 @@ def main():
                                  "speedup_qsa_vs_dense": d_ms / ms_step}
             del o
         if not args.no_cpu and world == 1:
+            import oracle  # test/baseline infrastructure only
+            threads = oracle.num_threads()
             v, secs, n = oracle_sample(w, x, args.cpu_rows, seed=12345)
+            v1, secs1, n1 = oracle_sample(w, x, max(8, args.cpu_rows // 8), seed=54321,
+                                          threads=1)
+            oracle.set_num_threads(threads)
             line["cpu_baseline"] = {
-                "value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                "value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                 "sample": f"{n} stratified query rows of {w.name} (index top-k + attention "
                           f"per row) plus pooling of the whole sequence, {secs:.1f} s wall; "
-                          f"rows/s extrapolated to tokens/s"}
+                          f"rows/s extrapolated to tokens/s",
+                "one_thread": {"value": v1, "unit": "tokens/s", "cores": 1,
+                               "sample": f"{n1} stratified rows, {secs1:.1f} s wall"}}
         if not args.no_extra:
             del run
             torch.cuda.empty_cache()
