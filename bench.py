@@ -212,17 +212,24 @@ class Prefill:
 
     def step(self, ev=None):
         q, w, x = self.qsa, self.w, self.x
+        nvtx = torch.cuda.nvtx
         if ev:
             ev[0].record(self.stream)
+        nvtx.range_push("qsa_pool")
         q.qsa_pool(x["k_idx"], self.kp, w.r, stream=self.stream)
+        nvtx.range_pop()
         if ev:
             ev[1].record(self.stream)
+        nvtx.range_push("qsa_index_topk")
         q.qsa_index_topk(x["q_idx"], x["w"], self.kp, self.sel, self.ws, w.r, w.budget,
                          stream=self.stream)
+        nvtx.range_pop()
         if ev:
             ev[2].record(self.stream)
+        nvtx.range_push("qsa_sparse_attn_prefill")
         q.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], self.sel, self.o, w.r, w.budget,
                                   w.scale, stream=self.stream)
+        nvtx.range_pop()
         if ev:
             ev[3].record(self.stream)
 
@@ -239,15 +246,19 @@ def flush_l2(buf):
 
 def time_prefill(run: Prefill, steps: int, warmup: int, world: int, device, flush=None,
                  clocks: Clocks | None = None):
+    nvtx = torch.cuda.nvtx
+    nvtx.range_push("warmup")
     for _ in range(warmup):
         run.step()
     torch.cuda.synchronize(device)
+    nvtx.range_pop()
     per = [events(4) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize(device)
     if clocks:
         clocks.start()
     t0, t1 = events(2)
+    nvtx.range_push("timed")
     t0.record(run.stream)
     for k in range(steps):
         if flush is not None:
@@ -255,6 +266,7 @@ def time_prefill(run: Prefill, steps: int, warmup: int, world: int, device, flus
         run.step(per[k])
     t1.record(run.stream)
     torch.cuda.synchronize(device)
+    nvtx.range_pop()
     barrier(world)
     clk = clocks.stop() if clocks else None
     total = t0.elapsed_time(t1)
