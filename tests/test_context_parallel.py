@@ -217,3 +217,41 @@ def test_context_parallel_kernels_equal_one_call_gpu():
     assert torch.equal(got["sel"], sel)
     assert torch.equal(got["o"].view(torch.int16), o.view(torch.int16))
     assert torch.equal(got["lse"], lse)
+
+
+# ------------------------------------------------------ a rank that dies --
+
+def _dying_worker(rank, world, port, q):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), OMP_NUM_THREADS="1")
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        os._exit(0)  # leaves between steps, before the all-gather, without a word
+    w = W_SMALL
+    x = synth.make_prefill(w, "cpu")
+    try:
+        cp.prefill_context_parallel(**_local(x, world, rank, w.r), r=w.r, budget=w.budget,
+                                    scale=w.scale, ops=OracleOps(w.r, w.budget, w.scale))
+        q.put((rank, "completed"))
+    except Exception as exc:  # the collective reports the missing rank
+        q.put((rank, type(exc).__name__))
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_fails_the_survivors_collective_instead_of_hanging():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:  # only processes this test started
+        p.kill()
+    assert not alive
+    rank, outcome = q.get(timeout=10)
+    assert rank == 0 and outcome != "completed"
