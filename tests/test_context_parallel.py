@@ -227,6 +227,7 @@ def _dying_worker(rank, world, port, q):
     sys.path.insert(0, ROOT)
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=10))
+    dist.barrier()  # both ranks are up
     if rank == 1:
         os._exit(0)  # leaves between steps, before the all-gather, without a word
     w = W_SMALL
@@ -237,6 +238,8 @@ def _dying_worker(rank, world, port, q):
         q.put((rank, "completed"))
     except Exception as exc:  # the collective reports the missing rank
         q.put((rank, type(exc).__name__))
+    q.close()
+    q.join_thread()  # the result reaches the parent before this process ends
     os._exit(0)
 
 
