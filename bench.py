@@ -393,6 +393,8 @@ def extra_prefill(qsa, name, device, peaks, flush):
     run = Prefill(qsa, w, x, device)
     total, kern, _ = time_prefill(run, 5, 3, 1, device, flush=flush)
     ms = total / 5
+    warm_total, _, _ = time_prefill(run, 5, 1, 1, device)  # no flush between steps
+    warm_ms = warm_total / 5
     o = torch.empty_like(x["q"])
     dense = time_call(lambda: qsa.qsa_dense_gqa_prefill(x["q"], x["k"], x["v"], o, w.scale),
                       run.stream, 2, 1, flush)
@@ -410,6 +412,7 @@ def extra_prefill(qsa, name, device, peaks, flush):
     except Exception as exc:  # no fused backend for this shape: report why
         sdpa = f"unavailable: {type(exc).__name__}"
     out = {"ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3), "kernels": rep,
+           "ms_per_step_warm": warm_ms,
            "torch_sdpa_dense_ms": sdpa,
            "dense_gqa_ms": dense,
            "dense_gqa_tflops": wk["dense_flops"] / (dense / 1e3) / 1e12,
