@@ -220,8 +220,13 @@ def test_index_invariants():
     assert sel[t].tolist() == [0, 1, 2, t // r]
 
 
-def test_needles_are_selected_tiny_workload():
-    w_ = synth.WORKLOADS["prefill-2k-tiny"]
+@pytest.mark.parametrize("name", ["prefill-2k-tiny", "prefill-32k", "prefill-128k"])
+def test_needles_are_selected_with_margin(name):
+    """Every planted needle of the workload is selected by the oracle with a
+    score margin above 1e-3 over the best block left out, so the GPU's selection
+    must keep it exactly (the generator plants needles strong enough for the
+    margin rule; this verifies that for the 2K, 32K and 128K workloads)."""
+    w_ = synth.WORKLOADS[name]
     x = synth.make_prefill(w_, "cpu")
     qi, ki = synth.bf16_bits(x["q_idx"]), synth.bf16_bits(x["k_idx"])
     wt = x["w"].numpy()
@@ -384,3 +389,51 @@ def test_needle_row_output_is_needle_value():
     o, _ = oracle.attn(bits["q"], bits["k"], bits["v"], w_.r, w_.scale, sel=sel, rows=rows)
     heads = np.arange(w_.Hkv) * w_.G             # the head each needle key copies
     np.testing.assert_allclose(o[:, heads], synth.NEEDLE_VALUE, atol=1e-3)
+
+
+# ------------------------------------------------------------ batch offsets --
+
+def test_batched_calls_equal_per_sequence_calls():
+    """A batch of sequences is the same computation as one call per sequence
+    (an identity of the definition: sequences never see each other).  The two
+    sequences get different indexer keys, pooled keys, K and V, so an oracle
+    that read sequence 0's pooled keys (or K/V) for sequence 1 -- a dropped
+    batch offset -- would fail here."""
+    rng = np.random.default_rng(5)
+    B, T, Hi, Di, Hq, Hkv, D, r, budget = 2, 96, 3, 16, 4, 2, 16, 4, 32
+    q_idx = _np_bf16(rng.standard_normal((B, T, Hi, Di)))
+    w = rng.random((B, T, Hi)).astype(np.float32)
+    k_idx = _np_bf16(rng.standard_normal((B, T, Di)))
+    q = _np_bf16(rng.standard_normal((B, T, Hq, D)))
+    k = _np_bf16(rng.standard_normal((B, T, Hkv, D)))
+    v = _np_bf16(rng.standard_normal((B, T, Hkv, D)))
+    kp = oracle.pool(k_idx, r)
+    assert not np.array_equal(kp[0], kp[1])
+    scale = 0.25
+    one = [(q_idx[b:b + 1], w[b:b + 1], kp[b:b + 1], q[b:b + 1], k[b:b + 1], v[b:b + 1])
+           for b in range(B)]
+
+    s2 = oracle.index_scores(q_idx, w, kp, r)
+    s1 = np.concatenate([oracle.index_scores(qi, wi, kpi, r) for qi, wi, kpi, *_ in one])
+    assert np.array_equal(s2, s1)
+
+    rows = np.array([5, 50, 95, T + 5, T + 50, T + 95], np.int64)
+    blocks = np.array([0, 7, 20, 0, 7, 20], np.int64)
+    p2 = oracle.score_pairs(q_idx, w, kp, rows, blocks)
+    p1 = np.concatenate([oracle.score_pairs(one[b][0], one[b][1], one[b][2], rows[3 * b:3 * b + 3] - b * T,
+                                            blocks[3 * b:3 * b + 3]) for b in range(B)])
+    assert np.array_equal(p2, p1)
+    # pairs of sequence 1 agree with its own dense score matrix, not sequence 0's
+    assert np.array_equal(p2[3:], s1[rows[3:], blocks[3:]])
+    assert not np.array_equal(p2[3:], s1[rows[3:] - T, blocks[3:]])
+
+    sel2, sc2, m2, c2 = oracle.index_topk(q_idx, w, kp, r, budget)
+    parts = [oracle.index_topk(qi, wi, kpi, r, budget) for qi, wi, kpi, *_ in one]
+    for a, i in ((sel2, 0), (sc2, 1), (m2, 2), (c2, 3)):
+        assert np.array_equal(a, np.concatenate([p[i] for p in parts]))
+
+    o2, l2 = oracle.attn(q, k, v, r, scale, sel=sel2)
+    for b in range(B):
+        o1, l1 = oracle.attn(one[b][3], one[b][4], one[b][5], r, scale, sel=parts[b][0])
+        assert np.array_equal(o2[b * T:(b + 1) * T], o1)
+        assert np.array_equal(l2[b * T:(b + 1) * T], l1)
