@@ -262,14 +262,17 @@ def time_prefill(run: Prefill, steps: int, warmup: int, world: int, device, flus
     t0.record(run.stream)
     for k in range(steps):
         if flush is not None:
-            flush_l2(flush)
+            flush_l2(flush)  # outside the step's own events
         run.step(per[k])
     t1.record(run.stream)
     torch.cuda.synchronize(device)
     nvtx.range_pop()
     barrier(world)
     clk = clocks.stop() if clocks else None
-    total = t0.elapsed_time(t1)
+    if flush is None:
+        total = t0.elapsed_time(t1)  # back-to-back steps
+    else:  # the steps' own event pairs, recorded after each flush
+        total = sum(e[0].elapsed_time(e[3]) for e in per)
     kern = {"pool": 0.0, "index_topk": 0.0, "sparse_attn": 0.0}
     for e in per:
         kern["pool"] += e[0].elapsed_time(e[1])
@@ -327,6 +330,30 @@ def time_call(fn, stream, reps, warm=1, flush=None):
     return sum(e[0].elapsed_time(e[1]) for e in evs) / reps
 
 
+def dense_peak(peaks, ms):
+    """bf16 peak for a dense call: the burst figure for a call timed alone, the
+    sustained one once the call itself runs for seconds."""
+    return peaks["bf16_tflops_sustained"] if ms >= 1000.0 else peaks["bf16_tflops"]
+
+
+def torch_sdpa_ms(x, w, stream, reps, warm, flush):
+    """torch's fused causal attention (flash / cuDNN) on the same tensors, with
+    the KV heads repeated to the query heads; context for the speed-up."""
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        qt = x["q"].transpose(1, 2)
+        kt = x["k"].repeat_interleave(w.G, dim=2).transpose(1, 2)
+        vt = x["v"].repeat_interleave(w.G, dim=2).transpose(1, 2)
+        with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.CUDNN_ATTENTION]):
+            ms = time_call(lambda: torch.nn.functional.scaled_dot_product_attention(
+                qt, kt, vt, is_causal=True, scale=w.scale), stream, reps, warm, flush)
+        del qt, kt, vt
+        torch.cuda.empty_cache()
+        return ms
+    except Exception as exc:  # no fused backend for this shape: report why
+        return f"unavailable: {type(exc).__name__}"
+
+
 def roof(achieved, peak, unit, bound, traffic=None):
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak if peak else None, "traffic": traffic}
@@ -347,23 +374,23 @@ def kernel_report(w, kern_ms, peaks):
                          "frac_tensor": wk["index_flops"] / s / 1e12 / tf,
                          "pairs_per_s": wk["index_pairs"] / s}
         elif name == "sparse_attn":
-            rep[name] = {"ms": ms, "GB/s": wk["attn_bytes"] / s / 1e9,
-                         "frac_hbm": wk["attn_bytes"] / s / 1e9 / hbm,
+            # the gathered K/V bytes are mostly served by L2 (selections overlap),
+            # so they are reported as a gather rate, not against the HBM peak;
+            # a DRAM fraction comes only from measured DRAM bytes
+            dram = MEASURED_TRAFFIC.get((w.name, name))
+            rep[name] = {"ms": ms, "gather_GB/s": wk["attn_bytes"] / s / 1e9,
                          "TFLOP/s": wk["attn_flops"] / s / 1e12,
-                         "frac_tensor": wk["attn_flops"] / s / 1e12 / tf}
+                         "frac_tensor": wk["attn_flops"] / s / 1e12 / tf,
+                         "dram_GB/s": dram / s / 1e9 if dram else None,
+                         "frac_hbm_measured": dram / s / 1e9 / hbm if dram else None}
     return rep, wk
 
 
-# DRAM bytes (read + write) per launch, from one single-pass ncu capture of the
-# same command's kernels (profiles/launches_prefill-1m.md gives the command and
-# the counters):  ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
-# dram__bytes_write.sum --clock-control none -k regex:"idx_tc|sparse_attn"
-# -s 4 -c 2 python bench.py --steps 1 --warmup 3 --no-extra --no-dense
-# --no-e2e --no-cpu.  Keyed by (workload, kernel); must be re-taken (or
-# removed) whenever that kernel changes.
+# DRAM bytes (read + write) per launch of a kernel, from a single-pass ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of that kernel in this
+# benchmark's own command; keyed by (workload, kernel).  An entry is valid only
+# for the kernel version it was taken on: remove it when the kernel changes.
 MEASURED_TRAFFIC = {
-    # ("prefill-1m", "index_topk"): re-take after the 32-bit bound selection
-    # (last capture, of the kernel before it: 3.87e9 + 12.01e9)
 }
 
 
@@ -377,7 +404,8 @@ def dominant_roofline(w, kern_ms, peaks, traffic=None):
         r = roof(wk["index_flops"] / s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s",
                  "tensor", traffic)
     elif name == "sparse_attn":
-        r = roof(wk["attn_bytes"] / s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm", traffic)
+        r = roof(wk["attn_flops"] / s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s",
+                 "tensor", traffic)
     else:
         r = roof(wk["pool_bytes"] / s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm", traffic)
     r["kernel"] = name
@@ -399,25 +427,15 @@ def extra_prefill(qsa, name, device, peaks, flush):
     dense = time_call(lambda: qsa.qsa_dense_gqa_prefill(x["q"], x["k"], x["v"], o, w.scale),
                       run.stream, 2, 1, flush)
     rep, wk = kernel_report(w, kern, peaks)
-    sdpa = None
-    try:  # torch's own fused attention (flash / cuDNN) on the same tensors, for context
-        from torch.nn.attention import SDPBackend, sdpa_kernel
-        qt = x["q"].transpose(1, 2)
-        kt = x["k"].repeat_interleave(w.G, dim=2).transpose(1, 2)
-        vt = x["v"].repeat_interleave(w.G, dim=2).transpose(1, 2)
-        with sdpa_kernel([SDPBackend.FLASH_ATTENTION, SDPBackend.CUDNN_ATTENTION]):
-            sdpa = time_call(lambda: torch.nn.functional.scaled_dot_product_attention(
-                qt, kt, vt, is_causal=True, scale=w.scale), run.stream, 2, 1, flush)
-        del qt, kt, vt
-    except Exception as exc:  # no fused backend for this shape: report why
-        sdpa = f"unavailable: {type(exc).__name__}"
+    sdpa = torch_sdpa_ms(x, w, run.stream, 2, 1, flush)
     out = {"ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3), "kernels": rep,
            "ms_per_step_warm": warm_ms,
            "torch_sdpa_dense_ms": sdpa,
            "dense_gqa_ms": dense,
            "dense_gqa_tflops": wk["dense_flops"] / (dense / 1e3) / 1e12,
-           "dense_frac_tensor": wk["dense_flops"] / (dense / 1e3) / 1e12 / peaks["bf16_tflops"],
-           "speedup_vs_dense": dense / ms, "l2": "flushed between iterations"}
+           "dense_frac_tensor": wk["dense_flops"] / (dense / 1e3) / 1e12 / dense_peak(peaks, dense),
+           "speedup_vs_torch_sdpa": sdpa / ms if isinstance(sdpa, float) else None,
+           "speedup_vs_own_dense": dense / ms, "l2": "flushed between iterations"}
     del x, run, o
     torch.cuda.empty_cache()
     return out
@@ -616,13 +634,23 @@ def run_reference(args, rank, world):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sum(secs) / len(secs), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, "oracle on a stratified row sample"),
+        "config": config_of(w, l2_label(w, x)),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def input_bytes(x) -> int:
+    return sum(x[n].numel() * x[n].element_size() for n in ("q", "k", "v", "q_idx", "k_idx", "w"))
+
+
+def l2_label(w, x) -> str:
+    b = input_bytes(x)
+    return ("L2 flushed between steps" if b < 4 * L2_BYTES else
+            f"inputs larger than L2 ({b / 1e9:.1f} GB per step)")
 
 
 def config_of(w, l2):
@@ -664,8 +692,7 @@ def main():
     w = synth.WORKLOADS[args.workload]
     seed = rank_seed(w, rank)
     x = synth.make_prefill(w, device, seed=seed)
-    in_bytes = sum(x[n].numel() * x[n].element_size()
-                   for n in ("q", "k", "v", "q_idx", "k_idx", "w"))
+    in_bytes = input_bytes(x)
     run = Prefill(qsa, w, x, device)
     flush = None
     if in_bytes < 4 * L2_BYTES:
@@ -683,8 +710,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": config_of(w, "flushed between steps" if flush is not None else
-                            f"inputs larger than L2 ({in_bytes / 1e9:.1f} GB per step)"),
+        "config": config_of(w, l2_label(w, x)),
         "roofline": roofline, "kernels": kern_rep,
         "gpu_launches": Prefill.LAUNCHES * args.steps,
         "clocks": clk,
@@ -707,12 +733,19 @@ def main():
                                           o[:, :4096].contiguous(), w.scale)
             d_ms = time_call(lambda: qsa.qsa_dense_gqa_prefill(x["q"], x["k"], x["v"], o, w.scale),
                              run.stream, 1, 0 if w.T >= 2**19 else 1, flush)
-            line["dense_gqa"] = {"ms": d_ms,
-                                 "tflops": wk["dense_flops"] / (d_ms / 1e3) / 1e12,
-                                 "frac_tensor": wk["dense_flops"] / (d_ms / 1e3) / 1e12
-                                 / peaks["bf16_tflops"],
-                                 "speedup_qsa_vs_dense": d_ms / ms_step}
             del o
+            torch.cuda.empty_cache()
+            sdpa = torch_sdpa_ms(x, w, run.stream, 1, 1, flush)
+            line["dense_gqa"] = {
+                "torch_sdpa_ms": sdpa,
+                "speedup_qsa_vs_torch_sdpa": sdpa / ms_step if isinstance(sdpa, float) else None,
+                "own_kernel_ms": d_ms,
+                "own_kernel_tflops": wk["dense_flops"] / (d_ms / 1e3) / 1e12,
+                "own_kernel_frac_tensor": wk["dense_flops"] / (d_ms / 1e3) / 1e12
+                / dense_peak(peaks, d_ms),
+                "speedup_qsa_vs_own_kernel": d_ms / ms_step,
+                "note": "torch SDPA (flash / cuDNN) is the main dense comparison; the "
+                        "library's own dense kernel is secondary"}
         if not args.no_cpu and world == 1:
             import oracle  # test/baseline infrastructure only
             threads = oracle.num_threads()

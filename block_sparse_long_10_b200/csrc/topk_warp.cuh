@@ -113,10 +113,12 @@ QSA_DEVICE uint64_t warp_kth_largest(const uint64_t *buf, int n, int K, uint32_t
     }
 }
 
-// The K-th largest of n 32-bit keys (1 <= K <= n; equal keys allowed: the
-// result is the K-th value counting multiplicity), same digit scheme.
-QSA_DEVICE uint32_t warp_kth_largest_u32(const uint32_t *buf, int n, int K, uint32_t *hist,
-                                         int lane) {
+// The K-th largest of n 32-bit (or 16-bit) keys (1 <= K <= n; equal keys
+// allowed: the result is the K-th value counting multiplicity), same digit
+// scheme.
+template <typename KeyT>
+QSA_DEVICE uint32_t warp_kth_largest_narrow(const KeyT *buf, int n, int K, uint32_t *hist,
+                                            int lane) {
     uint32_t mn = ~0u, mx = 0u;
     for (int i = lane; i < n; i += 32) {
         const uint32_t k = buf[i];
@@ -192,6 +194,11 @@ QSA_DEVICE uint32_t warp_kth_largest_u32(const uint32_t *buf, int n, int K, uint
         }
         top = shift - 1;
     }
+}
+
+QSA_DEVICE uint32_t warp_kth_largest_u32(const uint32_t *buf, int n, int K, uint32_t *hist,
+                                         int lane) {
+    return warp_kth_largest_narrow<uint32_t>(buf, n, K, hist, lane);
 }
 
 // Keep the keys >= kth (exactly K of them) at the front of buf; returns count.

@@ -151,3 +151,21 @@ def test_chunked_prefill_equals_one_shot():
     assert torch.equal(sel, sel1)
     assert torch.equal(o.view(torch.int16), o1.view(torch.int16))
     assert torch.equal(lse, lse1)
+
+
+@pytest.mark.parametrize("mode", ["signed", "one-head-zero"])
+def test_head_weights_of_any_sign(mode):
+    """The selection stays exact for head weights that are not a softmax:
+    N(0,1) weights (some negative) and weights with one head at zero.  The
+    prefill indexer's first pass uses a linear lower bound of the score whose
+    correction term is built from the negative weights; this checks that the
+    bound is valid in both cases (compared under the margin rule)."""
+    w = synth.Workload(f"w-{mode}", "prefill", 2, 3000, 8, 2, 128, 4, 64, 4, 512, 41, 4)
+    x = synth.make_prefill(w, DEV)
+    g = torch.Generator().manual_seed(43)
+    wt = torch.randn(w.B, w.T, w.Hi, generator=g)
+    if mode == "one-head-zero":
+        wt = wt.abs()
+        wt[..., 1] = 0.0
+    x["w"] = wt.to(DEV)
+    _check_prefill(w, x)

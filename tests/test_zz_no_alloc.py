@@ -1,9 +1,13 @@
 """The workspace-free decode attention (for callers that cannot allocate
-device memory where they run a decode step) against the workspace version.
+device memory where they run a decode step) against the workspace version and
+against the oracle.
 
 Collected last on purpose.  Two calls in a row through the C ABI must each
-match qsa_sparse_attn_decode on the same inputs within the parity tolerances,
-whether this file runs alone in a fresh process or after the other tests."""
+match qsa_sparse_attn_decode on the same inputs, and the oracle's attention
+over the same selection, within the parity tolerances, whether this file runs
+alone in a fresh process or after the other tests.  The entry point splits
+each selection into its own number of slices (about 512 slices per call),
+so the comparison with the oracle covers that slice configuration too."""
 import ctypes
 
 import numpy as np
@@ -11,6 +15,7 @@ import pytest
 import torch
 
 import block_sparse_long_10_b200 as qsa
+import oracle
 from block_sparse_long_10_b200 import synth
 from tests import parity
 
@@ -38,6 +43,11 @@ def test_noalloc_decode_matches_workspace_version_twice():
     wsa = qsa.workspace(qsa.qsa_sparse_attn_decode_workspace_size(B, w.Hq, w.D, 4, w.budget))
     qsa.qsa_sparse_attn_decode(x["q"], x["k_cache"], x["v_cache"], x["seqlens"], sel, o_ref,
                                wsa, 4, w.budget, w.scale, lse=lse_ref)
+    # the oracle's attention of every sequence over the same selection
+    pos0 = x["seqlens"].cpu().numpy().astype(np.int64) - 1
+    o_or, lse_or = oracle.attn(parity.bits(x["q"])[:, None], parity.bits(x["k_cache"]),
+                               parity.bits(x["v_cache"]), 4, w.scale, sel=sel.cpu().numpy(),
+                               q_pos0=pos0)
     for _ in range(2):
         o = torch.full_like(x["q"], float("nan"))
         lse = torch.full((B, w.Hq), float("nan"), dtype=torch.float32, device=DEV)
@@ -46,6 +56,8 @@ def test_noalloc_decode_matches_workspace_version_twice():
         torch.cuda.synchronize()
         _close(o, o_ref)
         assert (lse - lse_ref).abs().max().item() <= parity.LSE_ABS
+        parity.check_attention(oracle.bf16_bits_to_f64(parity.bits(o)).reshape(B, w.Hq, w.D),
+                               o_or, lse.cpu().numpy(), lse_or, "noalloc vs oracle")
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
