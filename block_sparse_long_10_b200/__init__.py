@@ -83,6 +83,10 @@ _SIGS = {
     "qsa_index_distill_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "qsa_index_distill": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
                                _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "qsa_index_distill_sparse_workspace_size": (_SZ, [_I, _I64, _I, _I, _I]),
+    "qsa_index_distill_sparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I,
+                                      _I, _I, _I, _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _SZ,
+                                      _VP]),
     "qsa_check_device_status": (_I, [_VP, _VP]),
     "qsa_status_string": (ctypes.c_char_p, [_I]),
     "qsa_version": (ctypes.c_char_p, []),
@@ -387,6 +391,45 @@ def qsa_index_distill(q, k, lse, q_idx, w, k_pooled, kl, dq_idx, dw, dk_pooled, 
     _call("qsa_index_distill", _ptr(q), _ptr(k), _ptr(lse), _ptr(q_idx), _ptr(w),
           _ptr(k_pooled), B, T, Hq, Hkv, D, Hi, Di, r, scale, _ptr(kl), _ptr(dq_idx), _ptr(dw),
           _ptr(dk_pooled), _ptr(dk_idx), _ptr(ws), ws.numel(), _stream(stream, q.device))
+
+
+def qsa_index_distill_sparse_workspace_size(B, T, Hkv, r=4, budget=2048) -> int:
+    return _size("qsa_index_distill_sparse_workspace_size", B, T, Hkv, r, budget)
+
+
+def qsa_index_distill_sparse(q, k, lse, sel, q_idx, w, k_pooled, kl, dq_idx, dw, dk_pooled,
+                             ws, r=4, budget=2048, scale=None, dk_idx=None, stream=None):
+    """Stage-2 indexer loss over the selection and the indexer gradients.
+
+    q [B,T,Hq,D], k [B,T,Hkv,D] bf16, lse [B,T,Hq] fp32 (the sparse attention's),
+    sel [B,T,budget//r] int32, q_idx [B,T,Hi,Di] bf16, w [B,T,Hi] fp32,
+    k_pooled [B,T//r,Di] bf16 -> kl [B,T], dq_idx [B,T,Hi,Di], dw [B,T,Hi],
+    dk_pooled [B,T//r,Di] and optionally dk_idx [B,T,Di], all fp32.
+    """
+    _need(q, _BF, "q", 4)
+    _need(k, _BF, "k", 4)
+    _need(lse, _F32, "lse", 3)
+    _need(sel, torch.int32, "sel", 3)
+    _need(q_idx, _BF, "q_idx", 4)
+    _need(w, _F32, "w", 3)
+    _need(k_pooled, _BF, "k_pooled", 3)
+    _need(kl, _F32, "kl", 2)
+    _need(dq_idx, _F32, "dq_idx", 4)
+    _need(dw, _F32, "dw", 3)
+    _need(dk_pooled, _F32, "dk_pooled", 3)
+    _need(dk_idx, _F32, "dk_idx", 3)
+    _need(ws, torch.uint8, "ws", 1)
+    B, T, Hq, D = q.shape
+    Hkv, Hi, Di = k.shape[2], q_idx.shape[2], q_idx.shape[3]
+    if tuple(sel.shape) != (B, T, budget // r):
+        raise ValueError("sel must be [B, T, budget//r]")
+    if tuple(k_pooled.shape) != (B, T // r, Di) or tuple(dk_pooled.shape) != (B, T // r, Di):
+        raise ValueError("k_pooled and dk_pooled must be [B, T//r, Di]")
+    scale = D ** -0.5 if scale is None else scale
+    _call("qsa_index_distill_sparse", _ptr(q), _ptr(k), _ptr(lse), _ptr(sel), _ptr(q_idx),
+          _ptr(w), _ptr(k_pooled), B, T, Hq, Hkv, D, Hi, Di, r, budget, scale, _ptr(kl),
+          _ptr(dq_idx), _ptr(dw), _ptr(dk_pooled), _ptr(dk_idx), _ptr(ws), ws.numel(),
+          _stream(stream, q.device))
 
 
 def qsa_check_device_status(ws, stream=None) -> int:

@@ -387,6 +387,44 @@ qsa_status_t qsa_index_distill(const qsa_bf16_t *q, const qsa_bf16_t *k, const f
                                                ws, static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------- stage-2 indexer loss --
+size_t qsa_index_distill_sparse_workspace_size(int B, int64_t T, int Hkv, int r, int budget) {
+    if (B < 1 || T < 0 || Hkv < 1 || r != 4 || budget < r || budget % r != 0) return SIZE_MAX;
+    return qsa::index_distill_sparse_ws_bytes(B, T, Hkv, budget / r);
+}
+
+qsa_status_t qsa_index_distill_sparse(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                      const float *lse, const int32_t *sel,
+                                      const qsa_bf16_t *q_idx, const float *w,
+                                      const qsa_bf16_t *k_pooled, int B, int64_t T, int Hq,
+                                      int Hkv, int D, int Hi, int Di, int r, int budget,
+                                      float scale, float *kl, float *dq_idx, float *dw,
+                                      float *dk_pooled, float *dk_idx, void *ws, size_t ws_bytes,
+                                      void *stream) {
+    if (B < 1 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || D < 1 || Hi < 1 || Di < 1 ||
+        r < 1 || budget < r || budget % r != 0 || !(scale == scale))
+        return QSA_ERR_INVALID_ARG;
+    if (T == 0) return QSA_OK;
+    const int64_t N = T / r;
+    if (!q || !k || !lse || !sel || !q_idx || !w || !kl || !dq_idx || !dw ||
+        (N > 0 && (!k_pooled || !dk_pooled)))
+        return QSA_ERR_INVALID_ARG;
+    const int kb = budget / r;
+    if (r != 4 || !supported_attn(Hq, Hkv, D) || !supported_indexer(Hi, Di) ||
+        kb > qsa::index_distill_sparse_max_entries())
+        return QSA_ERR_UNSUPPORTED_SHAPE;
+    if (!ws || ws_bytes < qsa::index_distill_sparse_ws_bytes(B, T, Hkv, kb) || !aligned16(ws))
+        return QSA_ERR_WORKSPACE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_idx) || !aligned16(k_pooled))
+        return QSA_ERR_INVALID_ARG;
+    int sms = 0;
+    qsa_status_t st = current_device(&sms);
+    if (st != QSA_OK) return st;
+    return from_cuda(qsa::launch_index_distill_sparse(
+        q, k, lse, sel, q_idx, w, k_pooled, B, T, Hq, Hkv, D, Hi, Di, kb, scale, kl, dq_idx, dw,
+        dk_pooled, dk_idx, ws, static_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------- status --
 qsa_status_t qsa_check_device_status(void *ws, void *stream) {
     if (!ws) return QSA_ERR_INVALID_ARG;

@@ -76,6 +76,17 @@ cudaError_t launch_index_distill(const uint16_t *q, const uint16_t *k, const flo
                                  float *kl, float *dq, float *dw, float *dkp, float *dk_idx,
                                  void *ws, cudaStream_t s);
 
+// Stage-2 indexer loss over the selection (sparse_distill.cu); the workspace holds
+// the sparse attention's mass per (KV group, row, selection entry) after the header.
+size_t index_distill_sparse_ws_bytes(int B, int64_t T, int Hkv, int kb);
+int index_distill_sparse_max_entries();
+cudaError_t launch_index_distill_sparse(const uint16_t *q, const uint16_t *k, const float *lse,
+                                        const int32_t *sel, const uint16_t *q_idx,
+                                        const float *w, const uint16_t *kp, int B, int64_t T,
+                                        int Hq, int Hkv, int D, int Hi, int Di, int kb,
+                                        float scale, float *kl, float *dq_idx, float *dw,
+                                        float *dkp, float *dk_idx, void *ws, cudaStream_t s);
+
 // Backward of the sparse prefill attention (sparse_bwd.cu); zeroes dk and dv first.
 cudaError_t launch_sparse_attn_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                         const int32_t *sel, const uint16_t *dout, int B,

@@ -306,6 +306,52 @@ QSA_API qsa_status_t qsa_index_distill(const qsa_bf16_t *q, const qsa_bf16_t *k,
                                        size_t ws_bytes, void *stream);
 
 /*
+ * Stage-2 indexer loss over the selection [ART: after the dense distillation,
+ * the second training stage trains the indexer together with the backbone so
+ * that the model adapts to the sparse attention pattern].  The pages give no
+ * formula; the reading: stage 1's KL restricted to each row's selected
+ * candidate blocks, with the layer's own sparse attention as the teacher.
+ *
+ * For query t of batch row b at position p = t, c = floor(p / r), and
+ * J(t) = { j in sel[b,t,:] : 0 <= j < c } (the selected blocks other than the
+ * forced own block):
+ *   a(t, j)  = sum over all Hq heads h and the r tokens u of block j of
+ *              exp(scale * q[b,t,h] . k[b,u,h/(Hq/Hkv)] - lse[b,t,h])
+ *              (lse: the sparse forward's, qsa_sparse_attn_prefill writes it)
+ *   pi(t, j) = a(t, j) / sum_{j' in J(t)} a(t, j')          (the teacher)
+ *   s(t, j)  = sum_h w[b,t,h] * max(0, q_idx[b,t,h,:] . k_pooled[b,j,:])
+ *   kl[b,t]  = KL(pi(t, .) || softmax_{j in J(t)} s(t, .)), 0 when |J(t)| < 2
+ * and the gradients of L = sum_{b,t} kl[b,t] as in qsa_index_distill, over J(t):
+ * g = softmax(s) - pi; dq_idx, dw per row; dk_pooled summed over rows (fp32
+ * atomics: the low-order bits vary from run to run); dk_idx = dk_pooled / r
+ * spread over each complete block's tokens, 0 on the trailing partial block.
+ *   q, k     [B, T, Hq, D] / [B, T, Hkv, D] bf16; lse [B, T, Hq] fp32 (natural log)
+ *   sel      [B, T, budget / r] int32 (qsa_index_topk's output for the same rows)
+ *   q_idx [B, T, Hi, Di] bf16, w [B, T, Hi] fp32, k_pooled [B, floor(T/r), Di] bf16
+ *            (NULL allowed when T < r)
+ *   kl [B, T], dq_idx [B, T, Hi, Di], dw [B, T, Hi], dk_pooled [B, floor(T/r), Di]
+ *            fp32 outputs (dk_pooled is overwritten, not accumulated into);
+ *            dk_idx [B, T, Di] fp32 or NULL
+ *   ws       at least qsa_index_distill_sparse_workspace_size(...) bytes, first
+ *            256 bytes zeroed once (status word); it holds the teacher's mass,
+ *            4 * Hkv * B * T * (budget / r) bytes
+ * A row whose teacher mass on its selected candidates underflows fp32 gets zero
+ * loss and gradients and records QSA_ERR_DEVICE.  T == 0 is a no-op.
+ * Constraints: r = 4, budget / r <= 1024, the attention shapes of
+ * qsa_sparse_attn_prefill, the indexer shapes of qsa_index_topk.
+ */
+QSA_API size_t qsa_index_distill_sparse_workspace_size(int B, int64_t T, int Hkv, int r,
+                                                       int budget);
+QSA_API qsa_status_t qsa_index_distill_sparse(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                              const float *lse, const int32_t *sel,
+                                              const qsa_bf16_t *q_idx, const float *w,
+                                              const qsa_bf16_t *k_pooled, int B, int64_t T,
+                                              int Hq, int Hkv, int D, int Hi, int Di, int r,
+                                              int budget, float scale, float *kl, float *dq_idx,
+                                              float *dw, float *dk_pooled, float *dk_idx,
+                                              void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Gated DeltaNet token mixing, the hybrid's other layers [ART: GDN keeps a
  * matrix state and, for each token, writes the error between the token's
  * information and what the memory holds for it, under a decay gate and a write
