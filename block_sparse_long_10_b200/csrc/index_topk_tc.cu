@@ -710,14 +710,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                     hit &= vm;
                 }
                 if (__any_sync(0xffffffffu, hit != 0)) {  // most tiles at long range
+                    // this lane's offset among the warp's survivors: the count's
+                    // bit planes by ballot (independent votes, no shuffle chain)
                     const int nl = __popc(hit);
-                    int incl = nl;
+                    const uint32_t lt = (1u << lane) - 1u;
+                    int excl = 0, tot = 0;
 #pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-                        if (lane >= off) incl += y;
+                    for (int bb = 0; (1 << bb) <= QPT; ++bb) {
+                        const uint32_t bal = __ballot_sync(0xffffffffu, (nl >> bb) & 1);
+                        excl += __popc(bal & lt) << bb;
+                        tot += __popc(bal) << bb;
                     }
-                    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+                    const int incl = excl + nl;
                     if (stg_n + tot > STG_ENT) flush();
                     if (tot > STG_ENT) {  // only with heavy ties: append directly
                         while (hit) {
