@@ -183,23 +183,30 @@ QSA_DEVICE float f2_sum(uint64_t p) {
 }
 
 // s = sum_h w_h * max(x_h, 0) in fp32, heads paired on the packed f32x2 pipe:
-// (w0 r0 + w2 r2) + (w1 r1 + w3 r3).  Both passes call this same function, so
-// a block's score is bit-identical in them.
+// (w0 r0 + w2 r2) + (w1 r1 + w3 r3).  The ReLU is taken on the FMA pipe as
+// x + |x| = 2 max(x, 0) (exact below half the float range), against halved
+// weights, so every product w_h max(x_h, 0) is the same fp32 value as with a
+// max instruction, which would run on the half-rate ALU pipe.  Both passes
+// call this same function, so a block's score is bit-identical in them.
+QSA_DEVICE float relu2(uint32_t v) {
+    const float x = __uint_as_float(v);
+    return x + fabsf(x);
+}
 template <int HI>
-QSA_DEVICE float score_of(const uint32_t *v, const float4 wq) {
-    const float r0 = fmaxf(__uint_as_float(v[0]), 0.f);
+QSA_DEVICE float score_of(const uint32_t *v, const float4 wh) {
+    const float r0 = relu2(v[0]);
     if constexpr (HI == 1) {
-        return wq.x * r0;
+        return wh.x * r0;
     } else {
-        const float r1 = fmaxf(__uint_as_float(v[1]), 0.f);
+        const float r1 = relu2(v[1]);
         uint64_t acc;
-        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(acc) : "l"(f2_pack(wq.x, wq.y)), "l"(f2_pack(r0, r1)));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(acc) : "l"(f2_pack(wh.x, wh.y)), "l"(f2_pack(r0, r1)));
         if constexpr (HI == 4) {
-            const float r2 = fmaxf(__uint_as_float(v[2]), 0.f);
-            const float r3 = fmaxf(__uint_as_float(v[3]), 0.f);
+            const float r2 = relu2(v[2]);
+            const float r3 = relu2(v[3]);
             asm("fma.rn.f32x2 %0, %1, %2, %0;"
                 : "+l"(acc)
-                : "l"(f2_pack(wq.z, wq.w)), "l"(f2_pack(r2, r3)));
+                : "l"(f2_pack(wh.z, wh.w)), "l"(f2_pack(r2, r3)));
         }
         return f2_sum(acc);
     }
@@ -530,7 +537,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int h = 0; h < HI; ++h) wv[h] = wr[h];
                 }
-                s_w[q] = make_float4(wv[0], wv[1], wv[2], wv[3]);
+                // halved: the scoring doubles the ReLU (exact both ways)
+                s_w[q] = make_float4(0.5f * wv[0], 0.5f * wv[1], 0.5f * wv[2], 0.5f * wv[3]);
                 s_c[q] = c;
                 s_cnt[q] = 0;
             }
@@ -557,12 +565,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int ch = 0; ch < NCH; ++ch) {
                         uint32_t v[CW];
                         sm100::tmem_ld16(taddr + CW * ch, v);
+                        if (!tail) {
 #pragma unroll
-                        for (int qq = 0; qq < CW / 2; ++qq) {
-                            const int x = ch * (CW / 2) + qq;
-                            const float lb =
-                                __uint_as_float(v[2 * qq]) + __uint_as_float(v[2 * qq + 1]);
-                            if (!tail || j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], lb);
+                            for (int qq = 0; qq < CW / 2; ++qq) {
+                                const int x = ch * (CW / 2) + qq;
+                                gm[x] = fmaxf(gm[x], __uint_as_float(v[2 * qq]) +
+                                                         __uint_as_float(v[2 * qq + 1]));
+                            }
+                        } else {
+#pragma unroll
+                            for (int qq = 0; qq < CW / 2; ++qq) {
+                                const int x = ch * (CW / 2) + qq;
+                                const float lb =
+                                    __uint_as_float(v[2 * qq]) + __uint_as_float(v[2 * qq + 1]);
+                                if (j < s_c[q0 + x]) gm[x] = fmaxf(gm[x], lb);
+                            }
                         }
                     }
                 } else {
@@ -692,9 +709,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                         for (int qq = 0; qq < CW / HI; ++qq) {
                             const int x = ch * (CW / HI) + qq;
                             const float s = score_of<HI>(v + qq * HI, s_w[q0 + x]);
-                            const bool keep = s > thp[x];
-                            hit = (hit << 1) | (uint32_t)keep;
-                            if (keep) scw[x * 32 + lane] = s;
+                            if (s > thp[x]) {
+                                hit |= 1u << (QPT - 1 - x);
+                                scw[x * 32 + lane] = s;
+                            }
                         }
                     }
                 }
@@ -714,12 +732,20 @@ __global__ void __launch_bounds__(THREADS, 1)
                     // bit planes by ballot (independent votes, no shuffle chain)
                     const int nl = __popc(hit);
                     const uint32_t lt = (1u << lane) - 1u;
-                    int excl = 0, tot = 0;
+                    int excl, tot;
+                    if (g.lb && !__any_sync(0xffffffffu, nl > 1)) {  // long rows: one per lane
+                        const uint32_t bal = __ballot_sync(0xffffffffu, nl);
+                        excl = __popc(bal & lt);
+                        tot = __popc(bal);
+                    } else {
+                        excl = 0;
+                        tot = 0;
 #pragma unroll
-                    for (int bb = 0; (1 << bb) <= QPT; ++bb) {
-                        const uint32_t bal = __ballot_sync(0xffffffffu, (nl >> bb) & 1);
-                        excl += __popc(bal & lt) << bb;
-                        tot += __popc(bal) << bb;
+                        for (int bb = 0; (1 << bb) <= QPT; ++bb) {
+                            const uint32_t bal = __ballot_sync(0xffffffffu, (nl >> bb) & 1);
+                            excl += __popc(bal & lt) << bb;
+                            tot += __popc(bal) << bb;
+                        }
                     }
                     const int incl = excl + nl;
                     if (stg_n + tot > STG_ENT) flush();
