@@ -456,12 +456,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ---------------------------------------------------- MMA issuer --
         if (lane == 0) {
             uint32_t it = 0;
+            // This thread shares its SM sub-partition with four epilogue warps,
+            // so the issue loop is kept short: the operand descriptors differ
+            // only in their start-address field (address >> 4, low 14 bits), so
+            // they are one constant high part and a 32-bit low part that the
+            // k-steps advance by 32 bytes (2 units) each.
+            const uint64_t desc_hi = sm100::smem_desc_kmajor(0, Lx::ROWB);
+            const uint32_t kp_lo = (smem_u32(sm + Lx::OFF_KP) >> 4) & 0x3FFFu;
+            const uint32_t q_lo = (smem_u32(sm + Lx::OFF_Q) >> 4) & 0x3FFFu;
             for (int i = 0;; ++i) {
                 const int tile = blockIdx.x + i * gridDim.x;
                 if (tile >= a.total_tiles) break;
                 const TileGeo g = tile_geo<QT, Lx::LB>(a, tile);
                 const int qb = i & 1;
-                const uint32_t b_base = smem_u32(sm + Lx::OFF_Q + qb * Lx::Q_TILE);
+                const uint32_t b_lo = q_lo + qb * (Lx::Q_TILE >> 4);
                 // one sweep of the pooled-key tiles against the buffer's operand
                 auto sweep = [&](bool op_ok, uint32_t idesc) {
                     for (int kt = 0; kt < g.n_kt; ++kt, ++it) {
@@ -474,13 +482,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                                                          abort_flag, a.wait_limit, a.ws);
                         if (!ok) continue;
                         sm100::tc_fence_after();
-                        const uint32_t a_base = smem_u32(sm + Lx::OFF_KP + s * Lx::KP_TILE);
+                        const uint32_t a_lo = kp_lo + s * (Lx::KP_TILE >> 4);
 #pragma unroll
                         for (int k = 0; k < KSTEPS; ++k)
-                            sm100::mma_bf16(tmem_base + tb * NCOL,
-                                            sm100::smem_desc_kmajor(a_base + k * 32, Lx::ROWB),
-                                            sm100::smem_desc_kmajor(b_base + k * 32, Lx::ROWB),
-                                            idesc, k > 0);
+                            sm100::mma_bf16(tmem_base + tb * NCOL, desc_hi | (a_lo + 2 * k),
+                                            desc_hi | (b_lo + 2 * k), idesc, k > 0);
                         sm100::mma_commit(&empty[s]);
                         sm100::mma_commit(&tfull[tb]);
                     }
