@@ -71,7 +71,7 @@ constexpr int CAP = 4096;        // candidate-list capacity per query (workspace
 constexpr int SELBUF = 1024;     // per selecting warp, u64 keys in shared memory
 constexpr int CHECK_EVERY = 16;  // pass-2 tiles between list-capacity checks
 constexpr int MAX_GROUPS = 16;   // group maxima per block lane and query
-constexpr int MAX_KEEP = 511;
+constexpr int MAX_KEEP = 511;    // the final sort network takes up to 512 keys
 constexpr int MAX_GRID = 160;
 constexpr int STG_ENT = 128;     // staged pass-2 survivors per epilogue warp
 
@@ -522,10 +522,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q0 = cq * QPT;                // first query of this thread
         const int p = lq * 32 + lane;           // block position within the tile
         const bool selw = e < SEL_WARPS;
-        uint32_t *hist = reinterpret_cast<uint32_t *>(sm + Lx::OFF_HIST) + (selw ? e : 0) * 256;
-        uint64_t *buf = reinterpret_cast<uint64_t *>(sm + Lx::OFF_BUF) + (size_t)(selw ? e : 0) * SELBUF;
         int sort_passes = 1;
         while (sort_passes < 4 && (a.n_blocks >> (8 * sort_passes)) > 0) ++sort_passes;
+        uint32_t *hist = reinterpret_cast<uint32_t *>(sm + Lx::OFF_HIST) + (selw ? e : 0) * 256;
+        uint64_t *buf = reinterpret_cast<uint64_t *>(sm + Lx::OFF_BUF) + (size_t)(selw ? e : 0) * SELBUF;
         uint32_t it = 0;
         for (int i = 0;; ++i) {
             const int tile = blockIdx.x + i * gridDim.x;
@@ -645,7 +645,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const int G = n_groups * MB;
                     if (K > 0 && G >= K && g.t0 + q < a.Tq) {
                         const uint16_t *src = gmax_g + (size_t)q * (MAX_GROUPS * MB);
-                        for (int x = lane; x < G; x += 32) kbuf[x] = src[x];
+                        for (int x = 8 * lane; x < G; x += 256)  // G is a multiple of 128
+                            cp_async16(smem_u32(kbuf + x), src + x, 16);
+                        cp_async_commit();
+                        cp_async_wait<0>();
                         __syncwarp();
                         // widen with zero low bits (rounds down); below the key of
                         // -inf lie only NaN patterns, so clamp there
@@ -822,11 +825,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const uint64_t kth = idx::warp_kth_largest(lst, n, K, hist, lane);
                         n = idx::warp_compact_ge(lst, n, kth, lane);
                     }
-                    for (int x = lane; x < n; x += 32) buf[x] = lst[x];
+                    // one asynchronous copy of the list (16-byte pieces, all in flight)
+                    for (int x = 2 * lane; x < n; x += 64)
+                        cp_async16(smem_u32(buf + x), lst + x, 16);
+                    cp_async_commit();
+                    cp_async_wait<0>();
                     __syncwarp();
                     int m = n;
                     if (n > K) {
-                        const uint64_t kth = idx::warp_kth_largest(buf, n, K, hist, lane);
+                        const uint64_t kth =
+                            idx::warp_kth_largest_bisect<SELBUF / 32>(buf, n, K, hist, lane);
                         m = idx::warp_compact_ge(buf, n, kth, lane);
                     }
                     // re-key as (block << 32 | score key) and sort by block

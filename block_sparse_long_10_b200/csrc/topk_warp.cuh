@@ -39,11 +39,22 @@ QSA_DEVICE uint64_t warp_max_u64(uint64_t v) {
 // then the answer).
 QSA_DEVICE uint64_t warp_kth_largest(const uint64_t *buf, int n, int K, uint32_t *hist,
                                      int lane) {
+    constexpr int U = 4;  // keys per lane loaded together (buf may be in global memory)
     uint64_t mn = ~0ull, mx = 0ull;
-    for (int i = lane; i < n; i += 32) {
-        const uint64_t k = buf[i];
-        mn = k < mn ? k : mn;
-        mx = k > mx ? k : mx;
+    for (int i0 = 0; i0 < n; i0 += 32 * U) {
+        uint64_t kk[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * 32 + lane;
+            kk[u] = i < n ? buf[i] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (i0 + u * 32 + lane < n) {
+                mn = kk[u] < mn ? kk[u] : mn;
+                mx = kk[u] > mx ? kk[u] : mx;
+            }
+        }
     }
     mn = warp_min_u64(mn);
     mx = warp_max_u64(mx);
@@ -58,12 +69,22 @@ QSA_DEVICE uint64_t warp_kth_largest(const uint64_t *buf, int n, int K, uint32_t
         const uint64_t hm = top >= 63 ? 0ull : (~0ull << (top + 1));
         for (int i = lane; i < 256; i += 32) hist[i] = 0;
         __syncwarp();
-        for (int i0 = 0; i0 < n; i0 += 32) {
-            const int i = i0 + lane;
-            const uint64_t k = i < n ? buf[i] : 0ull;
-            const bool m = i < n && (k & hm) == prefix;
-            const uint32_t d = (uint32_t)((shift >= 0 ? (k >> shift) : (k << -shift)) & 255u);
-            hist_add(hist, d, m, lane);
+        for (int i0 = 0; i0 < n; i0 += 32 * U) {
+            uint64_t kk[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * 32 + lane;
+                kk[u] = i < n ? buf[i] : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * 32 + lane;
+                const uint64_t k = kk[u];
+                const bool m = i < n && (k & hm) == prefix;
+                const uint32_t d =
+                    (uint32_t)((shift >= 0 ? (k >> shift) : (k << -shift)) & 255u);
+                hist_add(hist, d, m, lane);
+            }
         }
         __syncwarp();
         uint32_t local[8];
@@ -103,9 +124,16 @@ QSA_DEVICE uint64_t warp_kth_largest(const uint64_t *buf, int n, int K, uint32_t
         if ((int)cnt == want) {                          // bucket kept whole
             const uint64_t m2 = ~0ull << shift;
             uint64_t bmin = ~0ull;
-            for (int i = lane; i < n; i += 32) {
-                const uint64_t k = buf[i];
-                if ((k & m2) == prefix && k < bmin) bmin = k;
+            for (int i0 = 0; i0 < n; i0 += 32 * U) {
+                uint64_t kk[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = i0 + u * 32 + lane;
+                    kk[u] = i < n ? buf[i] : ~0ull;
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if ((kk[u] & m2) == prefix && kk[u] < bmin) bmin = kk[u];
             }
             return warp_min_u64(bmin);
         }
@@ -201,16 +229,84 @@ QSA_DEVICE uint32_t warp_kth_largest_u32(const uint32_t *buf, int n, int K, uint
     return warp_kth_largest_narrow<uint32_t>(buf, n, K, hist, lane);
 }
 
+// The K-th largest of n <= 32 R unique 64-bit keys in shared memory
+// (1 <= K <= n) with the high words held in registers: the K-th largest high
+// word t is built bit by bit from the top (keep a bit when at least K high
+// words are >= the prefix with it set), each step one predicated count per
+// register and one warp sum, with no shared-memory atomics.  High words above
+// t are all in; when the keys with high word t are exactly the rest, the K-th
+// key is the smallest of them; otherwise (equal scores across the cut) the
+// radix select above settles it.  Real keys have a nonzero high word (the
+// score key of any score >= -inf), so the zero padding never counts.
+template <int R>
+QSA_DEVICE uint64_t warp_kth_largest_bisect(const uint64_t *buf, int n, int K, uint32_t *hist,
+                                            int lane) {
+    uint32_t hi[R];
+    uint32_t mn = ~0u, mx = 0u;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int i = r * 32 + lane;
+        hi[r] = i < n ? (uint32_t)(buf[i] >> 32) : 0u;
+        if (i < n) {
+            mn = min(mn, hi[r]);
+            mx = max(mx, hi[r]);
+        }
+    }
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    uint32_t t;
+    if (mn == mx) {
+        t = mn;
+    } else {
+        const int top = 31 - __clz((int)(mn ^ mx));
+        t = top == 31 ? 0u : (mn & (~0u << (top + 1)));  // the bits every key shares
+#pragma unroll 1
+        for (int b = top; b >= 0; --b) {
+            const uint32_t c = t | (1u << b);
+            uint32_t cnt = 0;
+#pragma unroll
+            for (int r = 0; r < R; ++r) cnt += hi[r] >= c ? 1u : 0u;
+            if ((int)__reduce_add_sync(0xffffffffu, cnt) >= K) t = c;
+        }
+    }
+    uint32_t gt = 0, eq = 0, lo_min = ~0u;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        gt += hi[r] > t ? 1u : 0u;
+        if (hi[r] == t) {
+            ++eq;
+            lo_min = min(lo_min, (uint32_t)buf[r * 32 + lane]);
+        }
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
+    lo_min = __reduce_min_sync(0xffffffffu, lo_min);
+    if ((int)(gt + eq) == K) return ((uint64_t)t << 32) | lo_min;
+    return warp_kth_largest(buf, n, K, hist, lane);
+}
+
 // Keep the keys >= kth (exactly K of them) at the front of buf; returns count.
 QSA_DEVICE int warp_compact_ge(uint64_t *buf, int n, uint64_t kth, int lane) {
+    constexpr int U = 4;  // keys per lane loaded together (buf may be in global memory)
     int base = 0;
-    for (int i0 = 0; i0 < n; i0 += 32) {
-        const int i = i0 + lane;
-        const uint64_t k = (i < n) ? buf[i] : 0ull;
-        const bool keep = (i < n) && (k >= kth);
-        const uint32_t m = __ballot_sync(0xffffffffu, keep);
-        if (keep) buf[base + __popc(m & ((1u << lane) - 1u))] = k;
-        base += __popc(m);
+    for (int i0 = 0; i0 < n; i0 += 32 * U) {
+        uint64_t kk[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * 32 + lane;
+            kk[u] = i < n ? buf[i] : 0ull;
+        }
+        // every lane holds its batch before any lane writes (the writes only
+        // move keys to lower positions, which this batch has already read)
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * 32 + lane;
+            const bool keep = (i < n) && (kk[u] >= kth);
+            const uint32_t m = __ballot_sync(0xffffffffu, keep);
+            if (keep) buf[base + __popc(m & ((1u << lane) - 1u))] = kk[u];
+            base += __popc(m);
+        }
     }
     __syncwarp();
     return base;
