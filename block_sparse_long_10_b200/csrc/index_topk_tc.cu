@@ -104,6 +104,7 @@ struct L {
     static_assert(EPI_WARPS * QPT * 32 * 4 <= SEL_WARPS * SELBUF * 8, "pass-2 score park");
     static_assert(EPI_WARPS * MAX_GROUPS * MB * 2 <= SEL_WARPS * SELBUF * 8, "bound keys");
     static_assert((EPI_WARPS - SEL_WARPS) * 256 * 4 <= EPI_WARPS * STG_ENT * 8, "bound hists");
+    static_assert(SEL_WARPS * 512 * 4 <= EPI_WARPS * STG_ENT * 8, "sort hists");
     static constexpr int OFF_W = OFF_HIST + SEL_WARPS * 256 * 4;
     static constexpr int OFF_THR = OFF_W + QT * 16;
     static constexpr int OFF_C = OFF_THR + QT * 4;
@@ -522,8 +523,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q0 = cq * QPT;                // first query of this thread
         const int p = lq * 32 + lane;           // block position within the tile
         const bool selw = e < SEL_WARPS;
+        // 9-bit digits of the largest block id
         int sort_passes = 1;
-        while (sort_passes < 4 && (a.n_blocks >> (8 * sort_passes)) > 0) ++sort_passes;
+        while (sort_passes < 4 && ((a.n_blocks - 1) >> (9 * sort_passes)) > 0) ++sort_passes;
+        // the final sort's 512-bin histograms use the staging area, idle by then
+        uint32_t *hist9 = reinterpret_cast<uint32_t *>(sm + Lx::OFF_STGK) + (selw ? e : 0) * 512;
         uint32_t *hist = reinterpret_cast<uint32_t *>(sm + Lx::OFF_HIST) + (selw ? e : 0) * 256;
         uint64_t *buf = reinterpret_cast<uint64_t *>(sm + Lx::OFF_BUF) + (size_t)(selw ? e : 0) * SELBUF;
         uint32_t it = 0;
@@ -843,8 +847,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         buf[x] = ((uint64_t)(uint32_t)idx::key_block(k) << 32) | (k >> 32);
                     }
                     __syncwarp();
-                    const uint64_t *sorted = idx::warp_radix_sort_hi32(buf, buf + SELBUF / 2, m,
-                                                                       sort_passes, hist, lane);
+                    const uint64_t *sorted = idx::warp_radix_sort_hi32(
+                        buf, buf + SELBUF / 2, m, sort_passes, hist9, lane);
                     if (!aborted) {
                         int32_t *srow = a.sel + ((int64_t)g.b * a.Tq + t) * a.kb;
                         float *sc = a.sel_score ? a.sel_score + ((int64_t)g.b * a.Tq + t) * a.kb

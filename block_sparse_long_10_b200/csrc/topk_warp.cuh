@@ -312,28 +312,31 @@ QSA_DEVICE int warp_compact_ge(uint64_t *buf, int n, uint64_t kth, int lane) {
     return base;
 }
 
-// Stable LSD radix sort (8-bit digits) of m <= 1024 keys by their high 32
-// bits, which hold values below 2^(8*passes).  Ping-pongs between buf and
-// tmp; returns the buffer that holds the result.
+// Stable LSD radix sort (9-bit digits, 512-bin histogram: two passes cover
+// block ids below 2^18) of m <= 1024 keys by their high 32 bits, which hold
+// values below 2^(9*passes).  Ping-pongs between buf and tmp; returns the
+// buffer that holds the result.
 QSA_DEVICE uint64_t *warp_radix_sort_hi32(uint64_t *buf, uint64_t *tmp, int m, int passes,
-                                          uint32_t *hist, int lane) {
+                                            uint32_t *hist, int lane) {
+    constexpr int NB = 512, PER = NB / 32;
     const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll 1
     for (int p = 0; p < passes; ++p) {
-        const int sh = 32 + 8 * p;
-        for (int i = lane; i < 256; i += 32) hist[i] = 0;
+        const int sh = 32 + 9 * p;
+        for (int i = lane; i < NB; i += 32) hist[i] = 0;
         __syncwarp();
         for (int i0 = 0; i0 < m; i0 += 32) {
             const int i = i0 + lane;
-            const uint64_t k = i < m ? buf[i] : 0ull;
-            hist_add(hist, (uint32_t)(k >> sh) & 255u, i < m, lane);
+            const bool v = i < m;
+            const uint64_t k = v ? buf[i] : 0ull;
+            const uint32_t d = (uint32_t)(k >> sh) & (NB - 1);
+            hist_add(hist, d, v, lane);
         }
         __syncwarp();
-        // exclusive prefix sum over the 256 bins
-        uint32_t local[8], sum = 0;
+        uint32_t local[PER], sum = 0;
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            local[b] = hist[lane * 8 + b];
+        for (int b = 0; b < PER; ++b) {
+            local[b] = hist[lane * PER + b];
             sum += local[b];
         }
         uint32_t incl = sum;
@@ -345,8 +348,8 @@ QSA_DEVICE uint64_t *warp_radix_sort_hi32(uint64_t *buf, uint64_t *tmp, int m, i
         uint32_t run = incl - sum;
         __syncwarp();
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            hist[lane * 8 + b] = run;
+        for (int b = 0; b < PER; ++b) {
+            hist[lane * PER + b] = run;
             run += local[b];
         }
         __syncwarp();
@@ -354,11 +357,11 @@ QSA_DEVICE uint64_t *warp_radix_sort_hi32(uint64_t *buf, uint64_t *tmp, int m, i
             const int i = i0 + lane;
             const bool v = i < m;
             const uint64_t k = v ? buf[i] : 0ull;
-            const uint32_t d = (uint32_t)(k >> sh) & 255u;
+            const uint32_t d = (uint32_t)(k >> sh) & (NB - 1);
             // lanes holding the same digit: one ballot per digit bit
             uint32_t peers = __ballot_sync(0xffffffffu, v);
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
+            for (int b = 0; b < 9; ++b) {
                 const uint32_t bal = __ballot_sync(0xffffffffu, (d >> b) & 1u);
                 peers &= ((d >> b) & 1u) ? bal : ~bal;
             }
