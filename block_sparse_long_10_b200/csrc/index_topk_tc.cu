@@ -69,7 +69,8 @@ constexpr int SEL_WARPS = 8;     // epilogue warps that also run the selections
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr int CAP = 4096;        // candidate-list capacity per query (workspace)
 constexpr int SELBUF = 1024;     // per selecting warp, u64 keys in shared memory
-constexpr int CHECK_EVERY = 16;  // pass-2 tiles between list-capacity checks
+constexpr int CHECK_EVERY = 16;  // pass-2 tiles between list-capacity checks (even)
+static_assert(CHECK_EVERY % 2 == 0, "checks fall on the second tile of a pair");
 constexpr int MAX_GROUPS = 16;   // group maxima per block lane and query
 constexpr int MAX_KEEP = 511;    // the final sort network takes up to 512 keys
 constexpr int MAX_GRID = 160;
@@ -684,8 +685,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int x = 0; x < QPT; ++x) thp[x] = nextafterf(s_thr[q0 + x], -INFINITY);
             // this warp's survivor scores, [query x][lane]: the selection buffers
-            // are idle during pass 2 (16 warps x QPT x 32 floats fit in them)
-            float *scw = reinterpret_cast<float *>(sm + Lx::OFF_BUF) + e * (QPT * 32);
+            // are idle during pass 2.  Where two tiles' worth fit (16 warps x 2 x
+            // QPT x 32 floats), the survivors of a pair of tiles are staged
+            // together, halving the per-tile votes and their latency.
+            constexpr bool PAIR = 2 * EPI_WARPS * QPT * 32 * 4 <= SEL_WARPS * SELBUF * 8;
+            float *scw0 = reinterpret_cast<float *>(sm + Lx::OFF_BUF) + e * (QPT * 32);
+            float *scw1 = scw0 + (PAIR ? EPI_WARPS * QPT * 32 : 0);
+            uint32_t hit_p = 0;  // survivors of the pair's first tile, not yet staged
             // survivors are staged per warp in shared memory (no atomic on the
             // way) and moved to the query lists in batches, one entry per lane
             uint64_t *stg_key = reinterpret_cast<uint64_t *>(sm + Lx::OFF_STGK) + e * STG_ENT;
@@ -711,6 +717,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(lq * 32) << 16) + tb * NCOL + cq * (NCOL / 4);
                 uint32_t hit = 0;
+                float *scw = (kt & 1) ? scw1 : scw0;
                 {
                     constexpr int CW = 16;  // columns per load: 16 values live at a time
                     constexpr int NCH = NCOL / 4 / CW;
@@ -740,10 +747,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int x = 0; x < QPT; ++x) vm = (vm << 1) | (uint32_t)(j < s_c[q0 + x]);
                     hit &= vm;
                 }
-                if (__any_sync(0xffffffffu, hit != 0)) {  // most tiles at long range
+                // the pair's first tile waits for its second (list checks fall on
+                // second tiles: CHECK_EVERY is even)
+                if (PAIR && !(kt & 1) && kt + 1 != g.n_kt) {
+                    hit_p = hit;
+                    continue;
+                }
+                if (__any_sync(0xffffffffu, (hit | hit_p) != 0)) {  // most tiles at long range
                     // this lane's offset among the warp's survivors: the count's
                     // bit planes by ballot (independent votes, no shuffle chain)
-                    const int nl = __popc(hit);
+                    const int nl = __popc(hit) + __popc(hit_p);
                     const uint32_t lt = (1u << lane) - 1u;
                     int excl, tot;
                     if (g.lb && !__any_sync(0xffffffffu, nl > 1)) {  // long rows: one per lane
@@ -754,7 +767,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         excl = 0;
                         tot = 0;
 #pragma unroll
-                        for (int bb = 0; (1 << bb) <= QPT; ++bb) {
+                        for (int bb = 0; (1 << bb) <= (PAIR ? 2 * QPT : QPT); ++bb) {
                             const uint32_t bal = __ballot_sync(0xffffffffu, (nl >> bb) & 1);
                             excl += __popc(bal & lt) << bb;
                             tot += __popc(bal) << bb;
@@ -763,6 +776,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const int incl = excl + nl;
                     if (stg_n + tot > STG_ENT) flush();
                     if (tot > STG_ENT) {  // only with heavy ties: append directly
+                        while (hit_p) {
+                            const int b = 31 - __clz(hit_p);
+                            hit_p &= ~(1u << b);
+                            const int x = QPT - 1 - b;
+                            append(x, idx::make_key(scw0[x * 32 + lane], j - MB));
+                        }
                         while (hit) {
                             const int b = 31 - __clz(hit);
                             hit &= ~(1u << b);
@@ -771,6 +790,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                     } else {
                         int o = stg_n + incl - nl;
+                        while (hit_p) {  // the pair's first tile: parked in scw0
+                            const int b = 31 - __clz(hit_p);
+                            hit_p &= ~(1u << b);
+                            const int x = QPT - 1 - b;
+                            stg_key[o] = idx::make_key(scw0[x * 32 + lane], j - MB);
+                            stg_x[o] = (uint8_t)x;
+                            ++o;
+                        }
                         while (hit) {
                             const int b = 31 - __clz(hit);
                             hit &= ~(1u << b);
@@ -782,6 +809,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         stg_n += tot;
                     }
                 }
+                hit_p = 0;
                 // lists are checked every CHECK_EVERY tiles: a list below
                 // CAP - CHECK_EVERY * MB at a check cannot overflow before the next
                 if ((kt + 1) % CHECK_EVERY != 0 && kt + 1 != g.n_kt) continue;
