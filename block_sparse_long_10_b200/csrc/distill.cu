@@ -27,9 +27,10 @@
 //   2. rows_kernel: one warp per query row; pass 1 over its candidates gives
 //      Z, A and LSE (the row's loss), pass 2 forms dL/ds and accumulates dw
 //      and dq_idx.  Writes (Z, LSE) per row for kernel 3.
-//   3. dkp_kernel: one CTA per 32 blocks; streams the rows that see those
-//      blocks in tiles of 32 (indexer queries staged transposed in shared
-//      memory), recomputes dL/ds and accumulates dKp in registers: a fixed
+//   3. dkp_tc_kernel: one CTA per 32 blocks; streams the rows that see those
+//      blocks in tiles of 32, recomputes the head dot products on the tensor
+//      cores (mma.sync), forms dL/ds, and accumulates dKp = sum G^T Q_idx on
+//      the tensor cores with G split into bf16 high and low parts: a fixed
 //      summation order, no atomics.
 #include "qsa_common.cuh"
 #include "qsa_launch.h"
@@ -352,141 +353,192 @@ __global__ void __launch_bounds__(RW * 32)
 
 // ---------------------------------------------------------------- dKp --
 constexpr int JB = 32;  // blocks per CTA
-constexpr int DWARPS = 8;
-constexpr int DTHREADS = DWARPS * 32;
 constexpr int RT = 32;  // rows per tile
-constexpr int BPW = JB / DWARPS;  // blocks per warp
-constexpr int PAD = RT + 1;
 
+// dKp on the tensor cores.  Per CTA: JB pooled blocks; per tile of RT rows:
+//   A  d_h(t, j) = q_idx_h(t) . Kp(j) for the tile's 32 x 32 (row, block)
+//      pairs: one 16 x 8 tile per warp, mma.sync over Di (bf16 in, fp32 sum);
+//   B  per pair s, dL/ds and G_h = dL/ds w_h 1[d_h > 0] as in the rows
+//      kernel, written to shared memory as bf16 high and low parts
+//      (G = hi + lo to about 2^-17 relative);
+//   C  dKp[blocks x Di] += sum_h (G_h^hi + G_h^lo)^T Q_h, mma.sync with the
+//      rows as K; two 16 x 8 accumulator tiles per warp, in registers across
+//      all row tiles (a fixed summation order, no atomics).
+// Shared operand rows are padded by 16 bytes so that ldmatrix is free of bank
+// conflicts.
+constexpr int TCW = 8;  // warps
 template <int HI, int DI>
-struct DCfg {
-    static constexpr int QT = HI * DI * PAD;  // indexer queries, transposed: [h][k][t]
-    static constexpr int KPS = JB * DI;       // pooled keys of the tile
-    static constexpr int AT = JB * PAD;       // teacher mass [j][t]
-    static constexpr int WT = HI * RT;
-    static constexpr int FLOATS = QT + KPS + AT + WT + 2 * RT;
-    static constexpr int BYTES = FLOATS * 4;
+struct TcCfg {
+    static constexpr int KPSTR = DI * 2 + 16;       // [block][dim] bf16
+    static constexpr int QSTR = HI * DI * 2 + 16;   // [row][head][dim] bf16
+    static constexpr int GSTR = RT * 2 + 16;        // [head][hi/lo][block][row] bf16
+    static constexpr int OFF_KP = 0;
+    static constexpr int OFF_Q = OFF_KP + JB * KPSTR;
+    static constexpr int OFF_G = OFF_Q + RT * QSTR;
+    static constexpr int OFF_A = OFF_G + HI * 2 * JB * GSTR;   // [row][block] fp32
+    static constexpr int OFF_W = OFF_A + RT * JB * 4;          // [row][head] fp32
+    static constexpr int OFF_Z = OFF_W + RT * HI * 4;
+    static constexpr int OFF_L = OFF_Z + RT * 4;
+    static constexpr int BYTES = OFF_L + RT * 4;
+    static_assert(JB == 32 && RT == 32, "tile shape");
+    static_assert((DI / 8) % 2 == 0, "dims in pairs of n-tiles");
 };
 
 template <int HI, int DI>
-__global__ void __launch_bounds__(DTHREADS)
-    dkp_kernel(const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
-               const uint16_t *__restrict__ kp, const float *__restrict__ apart,
-               const float2 *__restrict__ stats, int B, int64_t T, int64_t N, int Hkv, int n_jt,
-               float *__restrict__ dkp, float *__restrict__ dk_idx) {
-    using C = DCfg<HI, DI>;
-    constexpr int DPL = DI / 32;
-    extern __shared__ __align__(16) float sm[];
-    float *qT = sm;
-    float *kpS = qT + C::QT;
-    float *aT = kpS + C::KPS;
-    float *wT = aT + C::AT;
-    float *Zs = wT + C::WT;
-    float *Ls = Zs + RT;
+__global__ void __launch_bounds__(TCW * 32)
+    dkp_tc_kernel(const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
+                  const uint16_t *__restrict__ kp, const float *__restrict__ apart,
+                  const float2 *__restrict__ stats, int B, int64_t T, int64_t N, int Hkv,
+                  int n_jt, float *__restrict__ dkp, float *__restrict__ dk_idx) {
+    using C = TcCfg<HI, DI>;
+    constexpr int KS = DI / 16;
+    constexpr int NT = DI / 8;  // dim n-tiles of the dKp tile
+    extern __shared__ __align__(128) uint8_t smem[];
+    float *sa = reinterpret_cast<float *>(smem + C::OFF_A);
+    float *sw = reinterpret_cast<float *>(smem + C::OFF_W);
+    float *sz = reinterpret_cast<float *>(smem + C::OFF_Z);
+    float *sl = reinterpret_cast<float *>(smem + C::OFF_L);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lr = lane >> 2, lc = lane & 3;
     const int jt = blockIdx.x % n_jt;
     const int64_t b = blockIdx.x / n_jt;
     const int64_t j0 = (int64_t)jt * JB;
     const int nj = (int)((N - j0) < JB ? (N - j0) : JB);
     const int64_t gstride = (int64_t)B * T * N;
 
-    for (int i = tid; i < C::KPS; i += DTHREADS) {
-        const int jj = i / DI, kk = i % DI;
-        kpS[i] = jj < nj ? __uint_as_float((uint32_t)kp[(b * N + j0 + jj) * DI + kk] << 16)
-                         : 0.f;
+    // the CTA's pooled keys (rows past nj zero)
+    for (int i = tid; i < JB * (DI / 8); i += TCW * 32) {
+        const int jj = i / (DI / 8), ch = i % (DI / 8);
+        cp_async16(smem_u32(smem + C::OFF_KP + jj * C::KPSTR + ch * 16),
+                   kp + (b * N + j0 + (jj < nj ? jj : 0)) * DI + ch * 8, jj < nj ? 16 : 0);
     }
-    float acc[BPW][DPL];
-#pragma unroll
-    for (int q4 = 0; q4 < BPW; ++q4)
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[q4][e] = 0.f;
+    cp_async_commit();
 
-    // rows that see block j0 as a candidate, and have at least two candidates
-    int64_t t_begin = (j0 + 1) * R;
+    // phase A/B: this warp's (row, block) tile; phase C: its two dKp tiles
+    const int am = warp >> 2, an = warp & 3;          // rows 16 am.., blocks 8 an..
+    const int cm = warp & 1, cn = (warp >> 1) * 2;    // blocks 16 cm.., dims 8 cn.. (2 tiles)
+    const bool cwork = cn < NT;  // Di = 32 has work for four warps only
+    float acc[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[u][e] = 0.f;
+
+    int64_t t_begin = (j0 + 1) * R;  // rows that see block j0 and have two candidates
     if (t_begin < 2 * R) t_begin = 2 * R;
+#pragma unroll 1
     for (int64_t t0 = t_begin; t0 < T; t0 += RT) {
-        __syncthreads();
-        for (int i = tid; i < RT * HI * DI; i += DTHREADS) {
-            const int tt = i / (HI * DI), hk = i % (HI * DI);
+        __syncthreads();  // the previous tile's operands are consumed
+        for (int i = tid; i < RT * (HI * DI / 8); i += TCW * 32) {
+            const int tt = i / (HI * DI / 8), ch = i % (HI * DI / 8);
             const int64_t t = t0 + tt;
-            qT[hk * PAD + tt] =
-                t < T ? __uint_as_float((uint32_t)q_idx[(b * T + t) * HI * DI + hk] << 16) : 0.f;
+            cp_async16(smem_u32(smem + C::OFF_Q + tt * C::QSTR + ch * 16),
+                       q_idx + (b * T + (t < T ? t : 0)) * HI * DI + ch * 8, t < T ? 16 : 0);
         }
-        for (int i = tid; i < RT * HI; i += DTHREADS) {
-            const int tt = i / HI, h = i % HI;
-            const int64_t t = t0 + tt;
-            wT[h * RT + tt] = t < T ? w[(b * T + t) * HI + h] : 0.f;
+        cp_async_commit();
+        for (int i = tid; i < RT * HI; i += TCW * 32) {
+            const int64_t t = t0 + i / HI;
+            sw[i] = t < T ? w[(b * T + t) * HI + i % HI] : 0.f;
         }
-        for (int i = tid; i < RT; i += DTHREADS) {
+        for (int i = tid; i < RT; i += TCW * 32) {
             const int64_t t = t0 + i;
             const float2 st = t < T ? stats[b * T + t] : make_float2(0.f, 0.f);
-            Zs[i] = st.x;
-            Ls[i] = st.y;
+            sz[i] = st.x;
+            sl[i] = st.y;
         }
-        for (int i = tid; i < RT * JB; i += DTHREADS) {
+        for (int i = tid; i < RT * JB; i += TCW * 32) {
             const int tt = i / JB, jj = i % JB;
             const int64_t t = t0 + tt, j = j0 + jj;
             float a = 0.f;
-            if (t < T && j < t / R)
+            if (t < T && jj < nj && j < t / R)
                 for (int gg = 0; gg < Hkv; ++gg) a += apart[gg * gstride + (b * T + t) * N + j];
-            aT[jj * PAD + tt] = a;
+            sa[i] = a;
         }
+        cp_async_wait<0>();
         __syncthreads();
 
-        const int64_t t = t0 + lane;
-        const int64_t ct = t < T ? t / R : 0;
-        const float Zt = Zs[lane], Lt = Ls[lane];
-        const float inv_z = Zt > 0.f ? 1.f / Zt : 0.f;
+        // ---- A: d_h for rows 16 am + (lr, lr + 8), blocks 8 an + (2 lc, 2 lc + 1)
+        float d[HI][4];
 #pragma unroll
-        for (int q4 = 0; q4 < BPW; ++q4) {
-            const int jl = warp * BPW + q4;
-            if (jl >= nj) break;
-            const int64_t j = j0 + jl;
-            float d[HI];
+        for (int h = 0; h < HI; ++h) {
 #pragma unroll
-            for (int h = 0; h < HI; ++h) d[h] = 0.f;
-#pragma unroll 8
-            for (int kk = 0; kk < DI; ++kk) {
-                const float kv = kpS[jl * DI + kk];
+            for (int e = 0; e < 4; ++e) d[h][e] = 0.f;
 #pragma unroll
-                for (int h = 0; h < HI; ++h) d[h] = fmaf(qT[(h * DI + kk) * PAD + lane], kv, d[h]);
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a0, a1, a2, a3, b0, b1;
+                const int ar = am * 16 + (lane & 15);
+                ldmatrix_x4(smem_u32(smem + C::OFF_Q + ar * C::QSTR + (h * DI + ks * 16) * 2 +
+                                     (lane >> 4) * 16),
+                            a0, a1, a2, a3);
+                const int br = an * 8 + (lane & 7);
+                ldmatrix_x2(smem_u32(smem + C::OFF_KP + br * C::KPSTR + ks * 32 +
+                                     ((lane >> 3) & 1) * 16),
+                            b0, b1);
+                mma_bf16_16816(d[h], a0, a1, a2, a3, b0, b1);
             }
+        }
+        // ---- B: dL/ds and G_h per pair, to shared memory as bf16 hi + lo
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = am * 16 + lr + (e >> 1) * 8;
+            const int jl = an * 8 + 2 * lc + (e & 1);
+            const int64_t t = t0 + rr, j = j0 + jl;
+            const int64_t ct = t < T ? t / R : 0;
+            const float Zt = sz[rr];
             float s = 0.f;
 #pragma unroll
-            for (int h = 0; h < HI; ++h) s = fmaf(wT[h * RT + lane], fmaxf(d[h], 0.f), s);
-            const bool valid = ct > j && ct >= 2 && Zt > 0.f;
-            const float gs = valid ? expf(s - Lt) - aT[jl * PAD + lane] * inv_z : 0.f;
-            float Gh[HI];
+            for (int h = 0; h < HI; ++h) s = fmaf(sw[rr * HI + h], fmaxf(d[h][e], 0.f), s);
+            const bool valid = jl < nj && ct > j && ct >= 2 && Zt > 0.f;
+            const float gs = valid ? expf(s - sl[rr]) - sa[rr * JB + jl] * (1.f / Zt) : 0.f;
 #pragma unroll
-            for (int h = 0; h < HI; ++h) Gh[h] = d[h] > 0.f ? gs * wT[h * RT + lane] : 0.f;
-#pragma unroll 4
-            for (int tt = 0; tt < RT; ++tt) {
-#pragma unroll
-                for (int h = 0; h < HI; ++h) {
-                    const float gh = __shfl_sync(FULL, Gh[h], tt);
-#pragma unroll
-                    for (int e = 0; e < DPL; ++e)
-                        acc[q4][e] = fmaf(gh, qT[(h * DI + lane * DPL + e) * PAD + tt], acc[q4][e]);
-                }
+            for (int h = 0; h < HI; ++h) {
+                const float g = d[h][e] > 0.f ? gs * sw[rr * HI + h] : 0.f;
+                const uint16_t hi = to_bf16_bits(g);
+                const uint16_t lo = to_bf16_bits(g - __uint_as_float((uint32_t)hi << 16));
+                uint16_t *gp = reinterpret_cast<uint16_t *>(smem + C::OFF_G) +
+                               ((h * 2) * JB + jl) * (C::GSTR / 2) + rr;
+                gp[0] = hi;
+                gp[JB * (C::GSTR / 2)] = lo;
             }
         }
+        __syncthreads();
+        // ---- C: dKp tiles (blocks 16 cm.., dims 8 (cn + u)..) += G^T Q
+        if (!cwork) continue;
+#pragma unroll
+        for (int h = 0; h < HI; ++h)
+#pragma unroll
+            for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+                for (int ks = 0; ks < RT / 16; ++ks) {
+                    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+                    const int gr = cm * 16 + (lane & 15);
+                    ldmatrix_x4(smem_u32(smem + C::OFF_G + ((h * 2 + hl) * JB + gr) * C::GSTR +
+                                         ks * 32 + (lane >> 4) * 16),
+                                a0, a1, a2, a3);
+                    const int qr = ks * 16 + (lane & 15);
+                    ldmatrix_x4_trans(smem_u32(smem + C::OFF_Q + qr * C::QSTR +
+                                               (h * DI + cn * 8) * 2 + (lane >> 4) * 16),
+                                      b0, b1, b2, b3);
+                    mma_bf16_16816(acc[0], a0, a1, a2, a3, b0, b1);
+                    mma_bf16_16816(acc[1], a0, a1, a2, a3, b2, b3);
+                }
     }
 
+    // rows 16 cm + lr (+8) are blocks, columns 8 (cn + u) + 2 lc (+1) are dims
+    if (!cwork) return;
 #pragma unroll
-    for (int q4 = 0; q4 < BPW; ++q4) {
-        const int jl = warp * BPW + q4;
-        if (jl >= nj) break;
-        const int64_t j = j0 + jl;
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) {
-            const int kk = lane * DPL + e;
-            dkp[(b * N + j) * DI + kk] = acc[q4][e];
+        for (int e = 0; e < 4; ++e) {
+            const int jl = cm * 16 + lr + (e >> 1) * 8;
+            const int kk = (cn + u) * 8 + 2 * lc + (e & 1);
+            if (jl >= nj) continue;
+            const int64_t j = j0 + jl;
+            dkp[(b * N + j) * DI + kk] = acc[u][e];
             if (dk_idx)
 #pragma unroll
-                for (int i = 0; i < R; ++i)
-                    dk_idx[(b * T + j * R + i) * DI + kk] = acc[q4][e] * (1.f / R);
+                for (int i = 0; i < R; ++i) dk_idx[(b * T + j * R + i) * DI + kk] = acc[u][e] * (1.f / R);
         }
-    }
 }
 
 template <int D, int G>
@@ -519,12 +571,12 @@ static cudaError_t launch_indexer_side(const uint16_t *q_idx, const float *w, co
         if (e != cudaSuccess) return e;
     }
     if (N > 0) {
-        using C = DCfg<HI, DI>;
-        auto kern = dkp_kernel<HI, DI>;
+        using C = TcCfg<HI, DI>;
+        auto kern = dkp_tc_kernel<HI, DI>;
         cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
         if (e != cudaSuccess) return e;
         const int n_jt = (int)((N + JB - 1) / JB);
-        kern<<<(unsigned)((int64_t)n_jt * B), DTHREADS, C::BYTES, s>>>(
+        kern<<<(unsigned)((int64_t)n_jt * B), TCW * 32, C::BYTES, s>>>(
             q_idx, w, kp, apart, stats, B, T, N, Hkv, n_jt, dkp, dk_idx);
         return cudaGetLastError();
     }
