@@ -24,9 +24,10 @@
 //      blocks' keys; each probability exp2(S log2e scale - lse log2e) is summed
 //      over the block's 4 keys and the KV group's G heads in registers and
 //      shuffles, and written once per (group, query, block) to the workspace.
-//   2. rows_kernel: one warp per query row; pass 1 over its candidates gives
-//      Z, A and LSE (the row's loss), pass 2 forms dL/ds and accumulates dw
-//      and dq_idx.  Writes (Z, LSE) per row for kernel 3.
+//   2. rows_tc_kernel: 32 query rows per CTA; pass 1 over their candidates
+//      (head dot products on mma.sync) gives Z, A and LSE (the rows' loss),
+//      pass 2 forms dL/ds, accumulates dw and dq_idx = sum G Kp on mma.sync.
+//      Writes (Z, LSE) per row for kernel 3.
 //   3. dkp_tc_kernel: one CTA per 32 blocks; streams the rows that see those
 //      blocks in tiles of 32, recomputes the head dot products on the tensor
 //      cores (mma.sync), forms dL/ds, and accumulates dKp = sum G^T Q_idx on
@@ -171,184 +172,6 @@ __global__ void __launch_bounds__(TTHREADS, 2)
         }
     }
     cp_async_wait<0>();
-}
-
-// --------------------------------------------------------------- rows --
-constexpr int RW = 8;  // rows (warps) per CTA
-
-template <int HI, int DI>
-__global__ void __launch_bounds__(RW * 32)
-    rows_kernel(const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
-                const uint16_t *__restrict__ kp, const float *__restrict__ apart, int B,
-                int64_t T, int64_t N, int Hkv, float *__restrict__ kl, float *__restrict__ dq,
-                float *__restrict__ dw, float *__restrict__ dk_idx, float2 *__restrict__ stats,
-                void *status) {
-    constexpr int DPL = DI / 32;  // dims per lane
-    __shared__ __align__(16) float qs_all[RW][HI * DI];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * RW + warp;
-    if (row >= (int64_t)B * T) return;
-    const int64_t b = row / T, t = row % T;
-    const int64_t c = t / R;
-    float *qs = qs_all[warp];
-
-    if (dk_idx && t >= N * R)  // tokens of the trailing partial block: no pooled key
-        for (int kk = lane; kk < DI; kk += 32) dk_idx[row * DI + kk] = 0.f;
-
-    auto zero_row = [&](float Z) {
-        for (int i = lane; i < HI * DI; i += 32) dq[row * HI * DI + i] = 0.f;
-        if (lane < HI) dw[row * HI + lane] = 0.f;
-        if (lane == 0) {
-            kl[row] = 0.f;
-            stats[row] = make_float2(Z, 0.f);
-        }
-    };
-    if (c < 2) {
-        zero_row(1.f);
-        return;
-    }
-
-    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(q_idx + row * HI * DI);
-    for (int i = lane; i < HI * DI / 2; i += 32) {
-        const uint32_t v = qrow[i];
-        qs[2 * i] = bf16_lo(v);
-        qs[2 * i + 1] = bf16_hi(v);
-    }
-    __syncwarp();
-    float wv[HI];
-#pragma unroll
-    for (int h = 0; h < HI; ++h) wv[h] = w[row * HI + h];
-    const uint16_t *kpb = kp + b * N * DI;
-    const float *arow = apart + (b * T + t) * N;
-    const int64_t gstride = (int64_t)B * T * N;
-
-    auto dots = [&](int64_t j, float (&d)[HI]) {
-#pragma unroll
-        for (int h = 0; h < HI; ++h) d[h] = 0.f;
-        const uint4 *kr = reinterpret_cast<const uint4 *>(kpb + j * DI);
-        // not unrolled: the row's queries stay in shared memory (broadcast reads)
-#pragma unroll 1
-        for (int c8 = 0; c8 < DI / 8; ++c8) {
-            const uint4 v = kr[c8];
-            const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-#pragma unroll
-            for (int h = 0; h < HI; ++h) {
-                const float4 qa = *reinterpret_cast<const float4 *>(qs + h * DI + c8 * 8);
-                const float4 qb = *reinterpret_cast<const float4 *>(qs + h * DI + c8 * 8 + 4);
-                d[h] = fmaf(qa.x, x[0], d[h]);
-                d[h] = fmaf(qa.y, x[1], d[h]);
-                d[h] = fmaf(qa.z, x[2], d[h]);
-                d[h] = fmaf(qa.w, x[3], d[h]);
-                d[h] = fmaf(qb.x, x[4], d[h]);
-                d[h] = fmaf(qb.y, x[5], d[h]);
-                d[h] = fmaf(qb.z, x[6], d[h]);
-                d[h] = fmaf(qb.w, x[7], d[h]);
-            }
-        }
-    };
-    auto score = [&](const float (&d)[HI]) {
-        float s = 0.f;
-#pragma unroll
-        for (int h = 0; h < HI; ++h) s = fmaf(wv[h], fmaxf(d[h], 0.f), s);
-        return s;
-    };
-    auto teacher = [&](int64_t j) {
-        float a = 0.f;
-        for (int gg = 0; gg < Hkv; ++gg) a += arow[gg * gstride + j];
-        return a;
-    };
-
-    // pass 1: Z, A and the scores' log-sum-exp
-    float m = -INFINITY, l = 0.f, Z = 0.f, A = 0.f;
-    for (int64_t j = lane; j < c; j += 32) {
-        float d[HI];
-        dots(j, d);
-        const float s = score(d);
-        const float a = teacher(j);
-        if (s > m) {
-            l = l * expf(m - s) + 1.f;
-            m = s;
-        } else {
-            l += expf(s - m);
-        }
-        Z += a;
-        if (a > 0.f) A += a * (logf(a) - s);
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-        const float m2 = __shfl_xor_sync(FULL, m, off);
-        const float l2 = __shfl_xor_sync(FULL, l, off);
-        const float mn = fmaxf(m, m2);
-        l = (mn == -INFINITY) ? 0.f : l * expf(m - mn) + l2 * expf(m2 - mn);
-        m = mn;
-        Z += __shfl_xor_sync(FULL, Z, off);
-        A += __shfl_xor_sync(FULL, A, off);
-    }
-    if (!(Z > 0.f)) {  // the teacher's candidate mass vanished in fp32
-        if (lane == 0) record_status(status, QSA_ERR_DEVICE);
-        zero_row(0.f);
-        return;
-    }
-    const float lse_s = m + logf(l);
-    const float inv_z = 1.f / Z;
-
-    // pass 2: dL/ds, then dw and dq_idx
-    float dwa[HI], acc[HI][DPL];
-#pragma unroll
-    for (int h = 0; h < HI; ++h) {
-        dwa[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
-    }
-    for (int64_t j0 = 0; j0 < c; j0 += 32) {
-        const int64_t j = j0 + lane;
-        float Gh[HI];
-        if (j < c) {
-            float d[HI];
-            dots(j, d);
-            const float gs = expf(score(d) - lse_s) - teacher(j) * inv_z;
-#pragma unroll
-            for (int h = 0; h < HI; ++h) {
-                dwa[h] = fmaf(gs, fmaxf(d[h], 0.f), dwa[h]);
-                Gh[h] = d[h] > 0.f ? gs * wv[h] : 0.f;
-            }
-        } else {
-#pragma unroll
-            for (int h = 0; h < HI; ++h) Gh[h] = 0.f;
-        }
-        const int n = (int)((c - j0) < 32 ? (c - j0) : 32);
-        for (int jj = 0; jj < n; ++jj) {
-            const uint16_t *kr = kpb + (j0 + jj) * DI + lane * DPL;
-            float x[DPL];
-            if constexpr (DPL == 2) {
-                const uint32_t v = *reinterpret_cast<const uint32_t *>(kr);
-                x[0] = bf16_lo(v);
-                x[1] = bf16_hi(v);
-            } else {
-                x[0] = __uint_as_float((uint32_t)kr[0] << 16);
-            }
-#pragma unroll
-            for (int h = 0; h < HI; ++h) {
-                const float gh = __shfl_sync(FULL, Gh[h], jj);
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(gh, x[e], acc[h][e]);
-            }
-        }
-    }
-#pragma unroll
-    for (int h = 0; h < HI; ++h) {
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) dq[(row * HI + h) * DI + lane * DPL + e] = acc[h][e];
-        float v = dwa[h];
-#pragma unroll
-        for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
-        if (lane == 0) dw[row * HI + h] = v;
-    }
-    if (lane == 0) {
-        kl[row] = A * inv_z - logf(Z) + lse_s;
-        stats[row] = make_float2(Z, lse_s);
-    }
 }
 
 // ---------------------------------------------------------------- dKp --
@@ -541,6 +364,313 @@ __global__ void __launch_bounds__(TCW * 32)
         }
 }
 
+// The rows' loss, dw and dq_idx on the tensor cores.  Per CTA: RT rows (one
+// sequence), swept twice over their candidate blocks in tiles of JB:
+//   pass 1  d_h on mma.sync (one 16 x 8 tile per warp, as in dkp_tc_kernel),
+//           s, the teacher mass a, and per row the scores' running log-sum-exp,
+//           Z and A, merged over lanes and warps at the end -> KL, (Z, LSE);
+//   pass 2  d_h again, dL/ds, dw_h += dL/ds max(0, d_h) per row, and
+//           G_h = dL/ds w_h 1[d_h > 0] to shared memory as bf16 high and low
+//           parts; dq_h[rows x Di] += G_h Kp on mma.sync, the accumulators of
+//           one (head, 16 rows, range of dims) per warp in registers.
+// Rows with fewer than two candidates get zeros, as in the definition.
+template <int HI, int DI>
+struct RtCfg {
+    static constexpr int NT = DI / 8;
+    static constexpr int TPW = HI * 2 * NT / TCW;   // dq n-tiles per warp
+    static_assert(TPW >= 1 && NT % TPW == 0, "dq tiles split evenly over the warps");
+    static constexpr int KPSTR = DI * 2 + 16;       // [block][dim] bf16
+    static constexpr int QSTR = HI * DI * 2 + 16;   // [row][head][dim] bf16
+    static constexpr int GSTR = JB * 2 + 16;        // [head][hi/lo][row][block] bf16
+    static constexpr int OFF_KP = 0;
+    static constexpr int OFF_Q = OFF_KP + JB * KPSTR;
+    static constexpr int OFF_G = OFF_Q + RT * QSTR;
+    static constexpr int OFF_A = OFF_G + HI * 2 * RT * GSTR;   // [row][block] fp32
+    static constexpr int OFF_W = OFF_A + RT * JB * 4;          // [row][head] fp32
+    static constexpr int OFF_R = OFF_W + RT * HI * 4;          // 4 warps x RT rows x 4 partials
+    static constexpr int OFF_S = OFF_R + 4 * RT * 4 * 4;       // per row: LSE, 1/Z, live flag
+    static constexpr int OFF_DW = OFF_S + RT * 4 * 4;          // 4 warps x RT rows x HI
+    static constexpr int BYTES = OFF_DW + 4 * RT * HI * 4;
+};
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(TCW * 32)
+    rows_tc_kernel(const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
+                   const uint16_t *__restrict__ kp, const float *__restrict__ apart, int B,
+                   int64_t T, int64_t N, int Hkv, int n_rt, float *__restrict__ kl,
+                   float *__restrict__ dq, float *__restrict__ dw, float *__restrict__ dk_idx,
+                   float2 *__restrict__ stats, void *status) {
+    using C = RtCfg<HI, DI>;
+    constexpr int KS = DI / 16;
+    extern __shared__ __align__(128) uint8_t smem[];
+    float *sa = reinterpret_cast<float *>(smem + C::OFF_A);
+    float *sw = reinterpret_cast<float *>(smem + C::OFF_W);
+    float *sred = reinterpret_cast<float *>(smem + C::OFF_R);
+    float *srow = reinterpret_cast<float *>(smem + C::OFF_S);
+    float *sdw = reinterpret_cast<float *>(smem + C::OFF_DW);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lr = lane >> 2, lc = lane & 3;
+    const int rt = n_rt - 1 - (int)(blockIdx.x % n_rt);  // longest rows first
+    const int64_t b = blockIdx.x / n_rt;
+    const int64_t t0 = (int64_t)rt * RT;
+    const int64_t t_end = t0 + RT < T ? t0 + RT : T;
+    const int64_t c_max = (t_end - 1) / R;  // candidates of the tile's last row
+    const int n_jt = (int)((c_max + JB - 1) / JB);
+    const int64_t gstride = (int64_t)B * T * N;
+
+    if (dk_idx)  // tokens of the trailing partial block: no pooled key
+        for (int i = tid; i < RT * DI; i += TCW * 32) {
+            const int64_t t = t0 + i / DI;
+            if (t < T && t >= N * R) dk_idx[(b * T + t) * DI + i % DI] = 0.f;
+        }
+    for (int i = tid; i < RT * (HI * DI / 8); i += TCW * 32) {
+        const int tt = i / (HI * DI / 8), ch = i % (HI * DI / 8);
+        const int64_t t = t0 + tt;
+        cp_async16(smem_u32(smem + C::OFF_Q + tt * C::QSTR + ch * 16),
+                   q_idx + (b * T + (t < T ? t : 0)) * HI * DI + ch * 8, t < T ? 16 : 0);
+    }
+    cp_async_commit();
+    for (int i = tid; i < RT * HI; i += TCW * 32) {
+        const int64_t t = t0 + i / HI;
+        sw[i] = t < T ? w[(b * T + t) * HI + i % HI] : 0.f;
+    }
+
+    const int am = warp >> 2, an = warp & 3;  // d tile: rows 16 am.., blocks 8 an..
+    // the candidate-block tile: pooled keys and the teacher mass
+    auto load_tile = [&](int jt) {
+        const int64_t jb0 = (int64_t)jt * JB;
+        for (int i = tid; i < JB * (DI / 8); i += TCW * 32) {
+            const int jj = i / (DI / 8), ch = i % (DI / 8);
+            const bool ok = jb0 + jj < c_max;
+            cp_async16(smem_u32(smem + C::OFF_KP + jj * C::KPSTR + ch * 16),
+                       kp + (b * N + (ok ? jb0 + jj : 0)) * DI + ch * 8, ok ? 16 : 0);
+        }
+        cp_async_commit();
+        for (int i = tid; i < RT * JB; i += TCW * 32) {
+            const int tt = i / JB, jj = i % JB;
+            const int64_t t = t0 + tt, j = jb0 + jj;
+            float a = 0.f;
+            if (t < T && j < t / R)
+                for (int gg = 0; gg < Hkv; ++gg) a += apart[gg * gstride + (b * T + t) * N + j];
+            sa[i] = a;
+        }
+        cp_async_wait<0>();
+    };
+    auto dots = [&](float (&d)[HI][4]) {
+#pragma unroll
+        for (int h = 0; h < HI; ++h) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[h][e] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a0, a1, a2, a3, b0, b1;
+                const int ar = am * 16 + (lane & 15);
+                ldmatrix_x4(smem_u32(smem + C::OFF_Q + ar * C::QSTR + (h * DI + ks * 16) * 2 +
+                                     (lane >> 4) * 16),
+                            a0, a1, a2, a3);
+                const int br = an * 8 + (lane & 7);
+                ldmatrix_x2(smem_u32(smem + C::OFF_KP + br * C::KPSTR + ks * 32 +
+                                     ((lane >> 3) & 1) * 16),
+                            b0, b1);
+                mma_bf16_16816(d[h], a0, a1, a2, a3, b0, b1);
+            }
+        }
+    };
+    auto score = [&](const float (&d)[HI][4], int e, int rr) {
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < HI; ++h) s = fmaf(sw[rr * HI + h], fmaxf(d[h][e], 0.f), s);
+        return s;
+    };
+
+    // ---- pass 1: the scores' log-sum-exp, Z and A per row ------------------
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, Zp[2] = {0.f, 0.f},
+          Ap[2] = {0.f, 0.f};
+#pragma unroll 1
+    for (int jt = 0; jt < n_jt; ++jt) {
+        __syncthreads();
+        load_tile(jt);
+        __syncthreads();
+        float d[HI][4];
+        dots(d);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = am * 16 + lr + (e >> 1) * 8;
+            const int64_t t = t0 + rr, j = (int64_t)jt * JB + an * 8 + 2 * lc + (e & 1);
+            if (t >= T || j >= t / R) continue;
+            const float s = score(d, e, rr);
+            const float a = sa[rr * JB + an * 8 + 2 * lc + (e & 1)];
+            const int k = e >> 1;
+            if (s > m[k]) {
+                l[k] = l[k] * expf(m[k] - s) + 1.f;
+                m[k] = s;
+            } else {
+                l[k] += expf(s - m[k]);
+            }
+            Zp[k] += a;
+            if (a > 0.f) Ap[k] += a * (logf(a) - s);
+        }
+    }
+    // merge over the quad's lanes, then over the four warps of each row half
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) {
+            const float m2 = __shfl_xor_sync(FULL, m[k], off);
+            const float l2 = __shfl_xor_sync(FULL, l[k], off);
+            const float mn = fmaxf(m[k], m2);
+            l[k] = (mn == -INFINITY) ? 0.f : l[k] * expf(m[k] - mn) + l2 * expf(m2 - mn);
+            m[k] = mn;
+            Zp[k] += __shfl_xor_sync(FULL, Zp[k], off);
+            Ap[k] += __shfl_xor_sync(FULL, Ap[k], off);
+        }
+        if (lc == 0) {
+            float *r4 = sred + ((an * RT) + am * 16 + lr + k * 8) * 4;
+            r4[0] = m[k];
+            r4[1] = l[k];
+            r4[2] = Zp[k];
+            r4[3] = Ap[k];
+        }
+    }
+    __syncthreads();
+    if (tid < RT) {
+        const int rr = tid;
+        const int64_t t = t0 + rr, row = b * T + t;
+        float M = -INFINITY, Lsum = 0.f, Z = 0.f, A = 0.f;
+        for (int wn = 0; wn < 4; ++wn) {
+            const float *r4 = sred + (wn * RT + rr) * 4;
+            const float mn = fmaxf(M, r4[0]);
+            Lsum = (mn == -INFINITY) ? 0.f : Lsum * expf(M - mn) + r4[1] * expf(r4[0] - mn);
+            M = mn;
+            Z += r4[2];
+            A += r4[3];
+        }
+        float live = 0.f, lse_s = 0.f, inv_z = 0.f;
+        if (t < T) {
+            if (t / R < 2) {
+                kl[row] = 0.f;
+                stats[row] = make_float2(1.f, 0.f);
+            } else if (!(Z > 0.f)) {  // the teacher's candidate mass vanished in fp32
+                record_status(status, QSA_ERR_DEVICE);
+                kl[row] = 0.f;
+                stats[row] = make_float2(0.f, 0.f);
+            } else {
+                lse_s = M + logf(Lsum);
+                inv_z = 1.f / Z;
+                live = 1.f;
+                kl[row] = A * inv_z - logf(Z) + lse_s;
+                stats[row] = make_float2(Z, lse_s);
+            }
+        }
+        srow[rr * 4 + 0] = lse_s;
+        srow[rr * 4 + 1] = inv_z;
+        srow[rr * 4 + 2] = live;
+    }
+
+    // ---- pass 2: dL/ds, dw and dq_idx --------------------------------------
+    // dq tiles of this warp: head qh, rows 16 qm.., dims 8 (qn0 + u)..
+    const int tile0 = warp * C::TPW;
+    const int qh = tile0 / (2 * C::NT), qm = (tile0 / C::NT) % 2, qn0 = tile0 % C::NT;
+    float acc[C::TPW][4];
+#pragma unroll
+    for (int u = 0; u < C::TPW; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[u][e] = 0.f;
+    float dwa[2][HI];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int h = 0; h < HI; ++h) dwa[k][h] = 0.f;
+#pragma unroll 1
+    for (int jt = 0; jt < n_jt; ++jt) {
+        __syncthreads();
+        load_tile(jt);
+        __syncthreads();
+        float d[HI][4];
+        dots(d);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = am * 16 + lr + (e >> 1) * 8;
+            const int jl = an * 8 + 2 * lc + (e & 1);
+            const int64_t t = t0 + rr, j = (int64_t)jt * JB + jl;
+            const bool valid = t < T && j < t / R && srow[rr * 4 + 2] > 0.f;
+            const float gs = valid ? expf(score(d, e, rr) - srow[rr * 4]) -
+                                         sa[rr * JB + jl] * srow[rr * 4 + 1]
+                                   : 0.f;
+#pragma unroll
+            for (int h = 0; h < HI; ++h) {
+                dwa[e >> 1][h] = fmaf(gs, fmaxf(d[h][e], 0.f), dwa[e >> 1][h]);
+                const float g = d[h][e] > 0.f ? gs * sw[rr * HI + h] : 0.f;
+                const uint16_t hi = to_bf16_bits(g);
+                const uint16_t lo = to_bf16_bits(g - __uint_as_float((uint32_t)hi << 16));
+                uint16_t *gp = reinterpret_cast<uint16_t *>(smem + C::OFF_G) +
+                               ((h * 2) * RT + rr) * (C::GSTR / 2) + jl;
+                gp[0] = hi;
+                gp[RT * (C::GSTR / 2)] = lo;
+            }
+        }
+        __syncthreads();
+        // dq_qh[rows 16 qm.., dims] += (G^hi + G^lo)[rows, blocks] Kp[blocks, dims]
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+            for (int ks = 0; ks < JB / 16; ++ks) {
+                uint32_t a0, a1, a2, a3;
+                const int gr = qm * 16 + (lane & 15);
+                ldmatrix_x4(smem_u32(smem + C::OFF_G + ((qh * 2 + hl) * RT + gr) * C::GSTR +
+                                     ks * 32 + (lane >> 4) * 16),
+                            a0, a1, a2, a3);
+                const int kr = ks * 16 + (lane & 15);
+                if constexpr (C::TPW == 1) {
+                    uint32_t b0, b1;
+                    ldmatrix_x2_trans(smem_u32(smem + C::OFF_KP + kr * C::KPSTR + qn0 * 16),
+                                      b0, b1);
+                    mma_bf16_16816(acc[0], a0, a1, a2, a3, b0, b1);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < C::TPW; u += 2) {
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4_trans(smem_u32(smem + C::OFF_KP + kr * C::KPSTR +
+                                                   (qn0 + u) * 16 + (lane >> 4) * 16),
+                                          b0, b1, b2, b3);
+                        mma_bf16_16816(acc[u], a0, a1, a2, a3, b0, b1);
+                        mma_bf16_16816(acc[u + 1], a0, a1, a2, a3, b2, b3);
+                    }
+                }
+            }
+    }
+
+    // dq: rows 16 qm + lr (+8), dims 8 (qn0 + u) + 2 lc (+1); rows with fewer
+    // than two candidates get zeros (G was zero for them)
+#pragma unroll
+    for (int u = 0; u < C::TPW; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int64_t t = t0 + qm * 16 + lr + (e >> 1) * 8;
+            if (t >= T) continue;
+            dq[((b * T + t) * HI + qh) * DI + (qn0 + u) * 8 + 2 * lc + (e & 1)] = acc[u][e];
+        }
+    // dw: over the quad's lanes, then the four warps of each row half
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int h = 0; h < HI; ++h) {
+            float v = dwa[k][h];
+            v += __shfl_xor_sync(FULL, v, 1);
+            v += __shfl_xor_sync(FULL, v, 2);
+            if (lc == 0) sdw[(an * RT + am * 16 + lr + k * 8) * HI + h] = v;
+        }
+    __syncthreads();
+    for (int i = tid; i < RT * HI; i += TCW * 32) {
+        const int rr = i / HI, h = i % HI;
+        const int64_t t = t0 + rr;
+        if (t >= T) continue;
+        float v = 0.f;
+        for (int wn = 0; wn < 4; ++wn) v += sdw[(wn * RT + rr) * HI + h];
+        dw[(b * T + t) * HI + h] = v;
+    }
+}
+
 template <int D, int G>
 static cudaError_t launch_teacher(const uint16_t *q, const uint16_t *k, const float *lse, int B,
                                   int64_t T, int Hkv, int64_t N, float scale, float *apart,
@@ -565,9 +695,14 @@ static cudaError_t launch_indexer_side(const uint16_t *q_idx, const float *w, co
                                        float2 *stats, void *status, cudaStream_t s) {
     const int64_t rows = (int64_t)B * T;
     if (rows > 0) {
-        rows_kernel<HI, DI><<<(unsigned)((rows + RW - 1) / RW), RW * 32, 0, s>>>(
-            q_idx, w, kp, apart, B, T, N, Hkv, kl, dq, dw, dk_idx, stats, status);
-        cudaError_t e = cudaGetLastError();
+        using C = RtCfg<HI, DI>;
+        auto kern = rows_tc_kernel<HI, DI>;
+        cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::BYTES);
+        if (e != cudaSuccess) return e;
+        const int n_rt = (int)((T + RT - 1) / RT);
+        kern<<<(unsigned)((int64_t)n_rt * B), TCW * 32, C::BYTES, s>>>(
+            q_idx, w, kp, apart, B, T, N, Hkv, n_rt, kl, dq, dw, dk_idx, stats, status);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (N > 0) {

@@ -73,6 +73,12 @@ QSA_DEVICE void ldmatrix_x2(uint32_t addr, uint32_t &r0, uint32_t &r1) {
                  : "r"(addr));
 }
 
+QSA_DEVICE void ldmatrix_x2_trans(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(addr));
+}
+
 // 8x8 b16 transpose within the warp's fragment layout.
 QSA_DEVICE uint32_t movmatrix_trans(uint32_t x) {
     uint32_t y;
