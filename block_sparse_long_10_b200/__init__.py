@@ -28,7 +28,8 @@ __all__ = [
     "qsa_dense_gqa_prefill",
     "qsa_dense_gqa_decode", "qsa_dense_gqa_decode_workspace_size",
     "qsa_index_distill", "qsa_index_distill_workspace_size", "qsa_sparse_attn_backward",
-    "qsa_gdn_prefill", "qsa_gdn_decode",
+    "qsa_gdn_prefill", "qsa_gdn_decode", "qsa_gdn_prefill_chunked",
+    "qsa_gdn_prefill_chunked_workspace_size",
     "qsa_check_device_status", "qsa_status_string", "qsa_version",
 ]
 
@@ -80,6 +81,9 @@ _SIGS = {
     "qsa_gdn_prefill": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _VP, _VP,
                              _VP]),
     "qsa_gdn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP, _VP]),
+    "qsa_gdn_prefill_chunked_workspace_size": (_SZ, [_I, _I64, _I, _I, _I]),
+    "qsa_gdn_prefill_chunked": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _VP,
+                                     _VP, _VP, _SZ, _VP]),
     "qsa_index_distill_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "qsa_index_distill": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _I, _I,
                                _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -340,6 +344,28 @@ def qsa_gdn_prefill(q, k, v, alpha, beta, o, state_out, state_in=None, stream=No
     B, T, H, dk = k.shape
     _call("qsa_gdn_prefill", _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in),
           B, T, H, dk, v.shape[3], _ptr(o), _ptr(state_out), _stream(stream, k.device))
+
+
+def qsa_gdn_prefill_chunked_workspace_size(B, T, H, dk, dv) -> int:
+    return _size("qsa_gdn_prefill_chunked_workspace_size", B, T, H, dk, dv)
+
+
+def qsa_gdn_prefill_chunked(q, k, v, alpha, beta, o, state_out, ws, state_in=None,
+                            stream=None):
+    """The same prefill in chunks of 64 tokens (chunk-parallel solves, state
+    products on the tensor cores); ws: a workspace of
+    qsa_gdn_prefill_chunked_workspace_size bytes."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, _BF, n, 4)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _need(t, _F32, n, 3)
+    _need(o, _F32, "o", 4)
+    _need(state_out, _F32, "state_out", 4)
+    _need(state_in, _F32, "state_in", 4)
+    B, T, H, dk = k.shape
+    _call("qsa_gdn_prefill_chunked", _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+          _ptr(state_in), B, T, H, dk, v.shape[3], _ptr(o), _ptr(state_out), _ptr(ws),
+          ws.numel() * ws.element_size(), _stream(stream, k.device))
 
 
 def qsa_gdn_decode(q, k, v, alpha, beta, state, o, stream=None):

@@ -339,6 +339,34 @@ qsa_status_t qsa_gdn_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k, const qsa
                                              state_out, static_cast<cudaStream_t>(stream)));
 }
 
+size_t qsa_gdn_prefill_chunked_workspace_size(int B, int64_t T, int H, int dk, int dv) {
+    if (B < 1 || T < 0 || H < 1 || !supported_gdn(dk, dv)) return SIZE_MAX;
+    return qsa::gdn_chunked_ws_bytes(B, T, H, dk, dv);
+}
+
+qsa_status_t qsa_gdn_prefill_chunked(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                     const qsa_bf16_t *v, const float *alpha, const float *beta,
+                                     const float *state_in, int B, int64_t T, int H, int dk,
+                                     int dv, float *o, float *state_out, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return QSA_ERR_INVALID_ARG;
+    if (!state_out || (T > 0 && (!q || !k || !v || !alpha || !beta || !o)))
+        return QSA_ERR_INVALID_ARG;
+    if (!supported_gdn(dk, dv)) return QSA_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(state_out) || (state_in && !aligned16(state_in)) ||
+        (T > 0 && (!aligned16(q) || !aligned16(k))))
+        return QSA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < qsa::gdn_chunked_ws_bytes(B, T, H, dk, dv) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return QSA_ERR_WORKSPACE;
+    int sms = 0;
+    qsa_status_t st = current_device(&sms);
+    if (st != QSA_OK) return st;
+    return from_cuda(qsa::launch_gdn_prefill_chunked(q, k, v, alpha, beta, state_in, B, T, H, dk,
+                                                     dv, o, state_out, ws,
+                                                     static_cast<cudaStream_t>(stream)));
+}
+
 qsa_status_t qsa_gdn_decode(const qsa_bf16_t *q, const qsa_bf16_t *k, const qsa_bf16_t *v,
                             const float *alpha, const float *beta, float *state, int B, int H,
                             int dk, int dv, float *o, void *stream) {

@@ -93,6 +93,14 @@ cudaError_t launch_sparse_attn_backward(const uint16_t *q, const uint16_t *k, co
                                         int64_t T, int Hq, int Hkv, int D, int kb, float scale,
                                         float *dq, float *dk, float *dv, cudaStream_t s);
 
+// Gated delta rule in chunks of 64 tokens (gdn_chunked.cu): chunk-parallel
+// triangular solves, then one CTA per (sequence, head) over its chunks.
+size_t gdn_chunked_ws_bytes(int B, int64_t T, int H, int dk, int dv);
+cudaError_t launch_gdn_prefill_chunked(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                       const float *alpha, const float *beta,
+                                       const float *state_in, int B, int64_t T, int H, int dk,
+                                       int dv, float *o, float *state_out, void *ws,
+                                       cudaStream_t s);
 // Gated delta rule (gdn.cu): exact recurrence, one CTA per (sequence, head).
 cudaError_t launch_gdn_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                const float *alpha, const float *beta, const float *state_in,

@@ -370,6 +370,29 @@ QSA_API qsa_status_t qsa_gdn_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k,
                                      const qsa_bf16_t *v, const float *alpha, const float *beta,
                                      const float *state_in, int B, int64_t T, int H, int dk,
                                      int dv, float *o, float *state_out, void *stream);
+/*
+ * The same prefill in chunks of 64 tokens [SUM: GDN, token mixing; the chunked
+ * form of the delta rule]: within a chunk, with gamma_t the product of the
+ * chunk's decay gates up to t and S0 the entering state, the writes
+ * u_t = beta_t (v_t - alpha_t S_{t-1} k_t) solve a unit lower-triangular system
+ * (I + A) U = diag(beta) V - diag(beta gamma) K S0^T, A_tj = beta_t
+ * (gamma_t / gamma_j) k_t.k_j; the outputs are diag(gamma) Q S0^T + P U,
+ * P_tj = (gamma_t / gamma_j) q_t.k_j (j <= t), and the next state gamma_last S0 +
+ * U^T diag(gamma_last / gamma) K.  The solves run for all chunks at once; the
+ * state products then run chunk after chunk on the tensor cores with fp32
+ * operands split into bf16 high and low parts (about 2^-16 relative per
+ * product).  Same arguments and layouts as qsa_gdn_prefill, plus a caller
+ * workspace of qsa_gdn_prefill_chunked_workspace_size bytes (256-byte aligned;
+ * per (sequence, head, chunk) the chunk's solve: 80.5 KiB at dk = dv = 128).
+ * Returns QSA_ERR_WORKSPACE if it is missing, too small or misaligned.
+ */
+QSA_API size_t qsa_gdn_prefill_chunked_workspace_size(int B, int64_t T, int H, int dk, int dv);
+QSA_API qsa_status_t qsa_gdn_prefill_chunked(const qsa_bf16_t *q, const qsa_bf16_t *k,
+                                             const qsa_bf16_t *v, const float *alpha,
+                                             const float *beta, const float *state_in, int B,
+                                             int64_t T, int H, int dk, int dv, float *o,
+                                             float *state_out, void *ws, size_t ws_bytes,
+                                             void *stream);
 QSA_API qsa_status_t qsa_gdn_decode(const qsa_bf16_t *q, const qsa_bf16_t *k,
                                     const qsa_bf16_t *v, const float *alpha, const float *beta,
                                     float *state, int B, int H, int dk, int dv, float *o,

@@ -177,6 +177,19 @@ def test_gdn_validation(lib):
     assert dec(B=0) == INVALID
     assert dec(st=_nullp()) == INVALID
     assert dec(dv=32) == UNSUPPORTED
+    # the chunked prefill: its workspace size, then the same checks plus the workspace
+    assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 64, 4, 128, 128) == 256 + 4 * 82432
+    assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 65, 4, 64, 64) == 256 + 2 * 4 * 49664
+    assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 64, 4, 96, 128) == SIZE_MAX
+    big = 1 << 24
+    chk = lambda **kw: lib.qsa_gdn_prefill_chunked(*dict(dict(
+        q=f, k=f, v=f, a=f, b=f, s0=None, B=1, T=64, H=4, dk=128, dv=128, o=f, s1=f, ws=f,
+        n=big), **kw).values(), s)
+    assert chk(H=0) == INVALID
+    assert chk(dk=96) == UNSUPPORTED
+    assert chk(ws=_nullp()) == WORKSPACE
+    assert chk(n=1000) == WORKSPACE
+    assert chk(ws=_fake(0x10010)) == WORKSPACE              # not 256-byte aligned
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
