@@ -400,6 +400,27 @@ def roof(achieved, peak, unit, bound, traffic=None):
             "frac": achieved / peak if peak else None, "traffic": traffic}
 
 
+def l2_read_gbs(qsa, device, mib=64, reps=40):
+    """L2-to-SM read bandwidth from the library's probe kernel (16-byte L2 loads
+    over a buffer that stays in L2), the denominator for gathers that L2 serves."""
+    buf = torch.ones(mib << 18, dtype=torch.float32, device=device)
+    sink = torch.zeros(1, dtype=torch.int32, device=device)
+    s = torch.cuda.current_stream(device)
+    for _ in range(2):
+        qsa.qsa_probe_l2_read(buf, reps, sink, stream=s)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(5):
+        e0, e1 = events(2)
+        e0.record(s)
+        qsa.qsa_probe_l2_read(buf, reps, sink, stream=s)
+        e1.record(s)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        best = ms if best is None else min(best, ms)
+    return (mib << 20) * reps / (best / 1e3) / 1e9
+
+
 def kernel_report(w, kern_ms, peaks):
     wk = prefill_work(w)
     hbm = peaks["hbm_gbs"]
@@ -423,7 +444,9 @@ def kernel_report(w, kern_ms, peaks):
                          "TFLOP/s": wk["attn_flops"] / s / 1e12,
                          "frac_tensor": wk["attn_flops"] / s / 1e12 / tf,
                          "dram_GB/s": dram / s / 1e9 if dram else None,
-                         "frac_hbm_measured": dram / s / 1e9 / hbm if dram else None}
+                         "frac_hbm_measured": dram / s / 1e9 / hbm if dram else None,
+                         "frac_l2_measured": (wk["attn_bytes"] / s / 1e9 / peaks["l2_gbs"]
+                                              if peaks.get("l2_gbs") else None)}
     return rep, wk
 
 
@@ -533,6 +556,37 @@ def extra_decode(qsa, device, peaks, flush):
         "launches_per_step": 4,
     }
     del x, kp
+    torch.cuda.empty_cache()
+    return out
+
+
+def extra_gdn(qsa, device, flush):
+    """The hybrid's other token mixer (gated delta rule) on one 16K-token sequence
+    with 16 heads of 128 x 128 state: the exact recurrence and the chunked form,
+    same inputs (unit keys, decay gates in [0.9, 1], write gates in [0, 1])."""
+    B, T, H, dk, dv = 1, 16384, 16, 128, 128
+    g = torch.Generator(device=device).manual_seed(7)
+    q = torch.randn(B, T, H, dk, generator=g, device=device).to(BF)
+    k = torch.randn(B, T, H, dk, generator=g, device=device)
+    k = (k / k.norm(dim=-1, keepdim=True)).to(BF)
+    v = torch.randn(B, T, H, dv, generator=g, device=device).to(BF)
+    a = 0.9 + 0.1 * torch.rand(B, T, H, generator=g, device=device)
+    b = torch.rand(B, T, H, generator=g, device=device)
+    s0 = torch.randn(B, H, dv, dk, generator=g, device=device) * 0.1
+    o1, o2 = (torch.empty(B, T, H, dv, device=device) for _ in range(2))
+    s1, s2 = (torch.empty(B, H, dv, dk, device=device) for _ in range(2))
+    ws = qsa.workspace(qsa.qsa_gdn_prefill_chunked_workspace_size(B, T, H, dk, dv), device)
+    st = torch.cuda.current_stream(device)
+    t_rec = time_call(lambda: qsa.qsa_gdn_prefill(q, k, v, a, b, o1, s1, state_in=s0, stream=st),
+                      st, 3, 1, flush)
+    t_chk = time_call(lambda: qsa.qsa_gdn_prefill_chunked(q, k, v, a, b, o2, s2, ws, state_in=s0,
+                                                          stream=st), st, 5, 1, flush)
+    diff = float((o1 - o2).abs().max() / o1.abs().max())
+    out = {"shape": {"B": B, "T": T, "H": H, "dk": dk, "dv": dv}, "recurrence_ms": t_rec,
+           "chunked_ms": t_chk, "speedup_chunked": t_rec / t_chk,
+           "tokens_per_s_chunked": B * T / (t_chk / 1e3),
+           "max_abs_diff_over_max": diff, "l2": "flushed between iterations"}
+    del ws
     torch.cuda.empty_cache()
     return out
 
@@ -732,6 +786,7 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     peaks = load_peaks()
+    peaks["l2_gbs"] = l2_read_gbs(qsa, device)
     w = synth.WORKLOADS[args.workload]
     seed = rank_seed(w, rank)
     x = synth.make_prefill(w, device, seed=seed)
@@ -755,6 +810,10 @@ def main():
         "data": "synthetic",
         "config": config_of(w, l2_label(w, x)),
         "roofline": roofline, "kernels": kern_rep,
+        "l2_probe": {"GB/s": peaks["l2_gbs"], "bytes": 64 << 20, "reps": 40,
+                     "note": "qsa_probe_l2_read: 16-byte L2 loads on all SMs over a 64 MiB "
+                             "buffer; the sparse attention's gather rate is also given as a "
+                             "fraction of it"},
         "gpu_launches": Prefill.LAUNCHES * args.steps,
         "clocks": clk,
     }
@@ -818,6 +877,10 @@ def main():
                 line["extra"]["distill-32k"] = extra_distill(qsa, device, peaks, fl)
             except Exception as exc:
                 line["extra"]["distill-32k"] = {"error": f"{type(exc).__name__}: {exc}"}
+            try:
+                line["extra"]["gdn-16k-h16"] = extra_gdn(qsa, device, fl)
+            except Exception as exc:
+                line["extra"]["gdn-16k-h16"] = {"error": f"{type(exc).__name__}: {exc}"}
         print(json.dumps(line), flush=True)
     barrier(world)
     if world > 1:

@@ -29,7 +29,7 @@ __all__ = [
     "qsa_dense_gqa_decode", "qsa_dense_gqa_decode_workspace_size",
     "qsa_index_distill", "qsa_index_distill_workspace_size", "qsa_sparse_attn_backward",
     "qsa_gdn_prefill", "qsa_gdn_decode", "qsa_gdn_prefill_chunked",
-    "qsa_gdn_prefill_chunked_workspace_size",
+    "qsa_gdn_prefill_chunked_workspace_size", "qsa_probe_l2_read",
     "qsa_check_device_status", "qsa_status_string", "qsa_version",
 ]
 
@@ -82,6 +82,7 @@ _SIGS = {
                              _VP]),
     "qsa_gdn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP, _VP]),
     "qsa_gdn_prefill_chunked_workspace_size": (_SZ, [_I, _I64, _I, _I, _I]),
+    "qsa_probe_l2_read": (_I, [_VP, _SZ, _I, _VP, _VP]),
     "qsa_gdn_prefill_chunked": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I64, _I, _I, _I, _VP,
                                      _VP, _VP, _SZ, _VP]),
     "qsa_index_distill_workspace_size": (_SZ, [_I, _I64, _I, _I]),
@@ -326,6 +327,15 @@ def qsa_sparse_attn_backward(q, k, v, sel, d_o, dq, dk, dv, r=4, budget=2048, sc
     _call("qsa_sparse_attn_backward", _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(d_o), B, T,
           Hq, k.shape[2], D, r, budget, scale, _ptr(dq), _ptr(dk), _ptr(dv),
           _stream(stream, q.device))
+
+
+# ---------------------------------------------------------- measurement aid --
+
+def qsa_probe_l2_read(buf, reps, sink, nbytes=None, stream=None):
+    """Reads the first nbytes (default: all) of the device buffer `buf` `reps`
+    times through L2; `sink` is a device int32 tensor the kernel may write."""
+    n = buf.numel() * buf.element_size() if nbytes is None else int(nbytes)
+    _call("qsa_probe_l2_read", _ptr(buf), n, int(reps), _ptr(sink), _stream(stream, buf.device))
 
 
 # ------------------------------------------------------------ Gated DeltaNet --

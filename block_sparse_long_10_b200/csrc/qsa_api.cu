@@ -318,6 +318,18 @@ qsa_status_t qsa_sparse_attn_backward(const qsa_bf16_t *q, const qsa_bf16_t *k,
                                                       static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------- measurement aid --
+qsa_status_t qsa_probe_l2_read(const void *buf, size_t bytes, int reps, void *sink,
+                               void *stream) {
+    if (!buf || !sink || reps < 1 || bytes < 16) return QSA_ERR_INVALID_ARG;
+    if (!aligned16(buf) || (reinterpret_cast<uintptr_t>(sink) & 3u) != 0) return QSA_ERR_INVALID_ARG;
+    int sms = 0;
+    qsa_status_t st = current_device(&sms);
+    if (st != QSA_OK) return st;
+    return from_cuda(qsa::launch_l2_read_probe(buf, bytes, reps, static_cast<uint32_t *>(sink),
+                                               sms, static_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------------- Gated DeltaNet --
 static bool supported_gdn(int dk, int dv) {
     return (dk == 64 || dk == 128) && (dv == 64 || dv == 128);

@@ -93,6 +93,9 @@ cudaError_t launch_sparse_attn_backward(const uint16_t *q, const uint16_t *k, co
                                         int64_t T, int Hq, int Hkv, int D, int kb, float scale,
                                         float *dq, float *dk, float *dv, cudaStream_t s);
 
+// Measurement aid (probe.cu): reads `bytes` of `buf` `reps` times through L2.
+cudaError_t launch_l2_read_probe(const void *buf, size_t bytes, int reps, uint32_t *sink,
+                                 int num_sms, cudaStream_t s);
 // Gated delta rule in chunks of 64 tokens (gdn_chunked.cu): chunk-parallel
 // triangular solves, then one CTA per (sequence, head) over its chunks.
 size_t gdn_chunked_ws_bytes(int B, int64_t T, int H, int dk, int dv);

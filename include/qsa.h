@@ -399,6 +399,18 @@ QSA_API qsa_status_t qsa_gdn_decode(const qsa_bf16_t *q, const qsa_bf16_t *k,
                                     void *stream);
 
 /*
+ * Measurement aid, not part of the attention path: reads the first `bytes` of
+ * the device buffer `buf` (16-byte aligned, >= 16 bytes) `reps` times with
+ * 16-byte loads cached in L2 only, on all SMs; `sink` is a device word the
+ * kernel may write (to keep its loads live).  Timed around with events over a
+ * buffer that fits in L2, it gives the L2-to-SM read bandwidth that kernels
+ * with L2-resident sources are rated against.  Bytes read = bytes * reps
+ * (rounded down to 16-byte units).
+ */
+QSA_API qsa_status_t qsa_probe_l2_read(const void *buf, size_t bytes, int reps, void *sink,
+                                       void *stream);
+
+/*
  * Synchronises `stream`, reads the status word kernels recorded at the start
  * of `ws`, clears it, and returns it (QSA_OK if nothing was recorded).  The
  * word is sticky: it keeps the first error recorded by any call that used
