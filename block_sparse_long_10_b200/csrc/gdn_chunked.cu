@@ -17,12 +17,13 @@
 //                   products, the triangular solve for [Ut | W] by forward
 //                   substitution (fp32 on CUDA cores), written to the
 //                   workspace (W and P as bf16 high + low parts);
-//   gdn_chunk_scan  one CTA per (sequence, head) walks its chunks in order with
-//                   the state in registers; the three state products
-//                   (W S0^T, Q S0^T, U^T diag(g) K) and P U run on mma.sync
-//                   with every fp32 operand split into bf16 high and low parts
-//                   (hi.hi + hi.lo + lo.hi, about 2^-16 relative), so the
-//                   result keeps fp32-level accuracy.
+//   gdn_chunk_scan  per (sequence, head), VS = 16 rows of the state per CTA
+//                   (the rows are independent: U, O and the state update of a
+//                   row slice need only that slice), each CTA walking its chunks
+//                   in order with its rows of the state in registers; the state
+//                   products (W S0^T, Q S0^T, U^T diag(g) K) and P U run on
+//                   mma.sync with every fp32 operand split into bf16 high and
+//                   low parts (hi.hi + hi.lo + lo.hi, about 2^-16 relative).
 // Tokens past the end of the sequence enter the last chunk as alpha = 1,
 // beta = 0 and zero vectors: they change nothing.
 #include "qsa_common.cuh"
@@ -41,8 +42,9 @@ struct Ws {  // per (sequence, head, chunk) record in the workspace, bytes
     static constexpr size_t U = (size_t)C * DV * 4;   // Ut (fp32)
     static constexpr size_t P = (size_t)C * C * 2;    // each of hi, lo (bf16)
     static constexpr size_t OFF_WH = 0, OFF_WL = W, OFF_U = 2 * W, OFF_PH = 2 * W + U,
-                            OFF_PL = OFF_PH + P, OFF_G = OFF_PL + P;   // gamma[C], g[C]
-    static constexpr size_t BYTES = (OFF_G + 2 * C * 4 + 255) / 256 * 256;
+                            OFF_PL = OFF_PH + P, OFF_G = OFF_PL + P,   // gamma[C], g[C]
+                            OFF_KH = OFF_G + 2 * C * 4, OFF_KL = OFF_KH + W;  // g_t k_t hi, lo
+    static constexpr size_t BYTES = (OFF_KL + W + 255) / 256 * 256;
 };
 
 QSA_DEVICE void split_bf16(float x, uint16_t &hi, uint16_t &lo) {
@@ -170,33 +172,42 @@ __global__ void __launch_bounds__(THREADS)
         g[tid] = expf(ell[tid]);                  // gamma_t
         g[C + tid] = expf(ell[C - 1] - ell[tid]); // gamma_{C-1} / gamma_t
     }
+    for (int i = tid; i < C * DK; i += THREADS) {  // g_t k_t, the state update's operand
+        const int t = i / DK, d = i % DK;
+        uint16_t kh, kl;
+        split_bf16(expf(ell[C - 1] - ell[t]) * Ks[t * (DK + 1) + d], kh, kl);
+        reinterpret_cast<uint16_t *>(rec + W::OFF_KH)[t * DK + d] = kh;
+        reinterpret_cast<uint16_t *>(rec + W::OFF_KL)[t * DK + d] = kl;
+    }
 }
 
 // ---------------------------------------------------------------- scan --
+constexpr int VS = 16;  // state rows (value dims) per scan CTA
+
 template <int DK, int DV>
 struct ScanCfg {
-    static constexpr int SSTR = DK * 2 + 16;  // state hi/lo [DV][DK] bf16, padded rows
+    static constexpr int SSTR = DK * 2 + 16;  // state hi/lo [VS][DK] bf16, padded rows
     static constexpr int WSTR = DK * 2 + 16;  // W hi/lo, Q, gK hi/lo [C][DK] bf16
     static constexpr int PSTR = C * 2 + 16;   // P hi/lo [C][C] bf16
-    static constexpr int USTR = DV * 2 + 16;  // U hi/lo [C][DV] bf16
+    static constexpr int USTR = VS * 2 + 16;  // U hi/lo [C][VS] bf16
+    static constexpr int NSL = DV / VS;       // CTAs per (sequence, head)
     static constexpr int OFF_SH = 0;
-    static constexpr int OFF_SL = OFF_SH + DV * SSTR;
-    static constexpr int OFF_WH = OFF_SL + DV * SSTR;
-    static constexpr int OFF_WL = OFF_WH + C * WSTR;
-    static constexpr int OFF_Q = OFF_WL + C * WSTR;
-    static constexpr int OFF_KH = OFF_Q + C * WSTR;
-    static constexpr int OFF_KL = OFF_KH + C * WSTR;
-    static constexpr int OFF_PH = OFF_KL + C * WSTR;
-    static constexpr int OFF_PL = OFF_PH + C * PSTR;
-    static constexpr int OFF_UH = OFF_PL + C * PSTR;
+    static constexpr int OFF_SL = OFF_SH + VS * SSTR;
+    static constexpr int OFF_UH = OFF_SL + VS * SSTR;
     static constexpr int OFF_UL = OFF_UH + C * USTR;
-    static constexpr int OFF_GM = OFF_UL + C * USTR;   // gamma [C] fp32
-    static constexpr int BYTES = OFF_GM + C * 4;
+    static constexpr int OFF_ST = OFF_UL + C * USTR;   // two stages of a chunk's operands
+    // within a stage
+    static constexpr int WH = 0, WL = WH + C * WSTR, Q = WL + C * WSTR, KH = Q + C * WSTR,
+                         KL = KH + C * WSTR, PH = KL + C * WSTR, PL = PH + C * PSTR,
+                         GM = PL + C * PSTR;            // gamma [C] fp32
+    static constexpr int STAGE = GM + C * 4;
+    static constexpr int BYTES = OFF_ST + 2 * STAGE;
     // state tiles (rows v, columns k): MT x NTS tiles of 16 x 8 over 8 warps
-    static constexpr int MT = DV / 16, NTS = DK / 8, WPM = 8 / MT, NPW = NTS / WPM;
-    // U / O tiles (rows t, columns v): 4 x DV/8 tiles, DV/16 per warp
-    static constexpr int NU = DV / 16;
+    static constexpr int MT = VS / 16, NTS = DK / 8, WPM = 8 / MT, NPW = NTS / WPM;
+    // U / O tiles (rows t, columns v): 4 x VS/8 tiles, VS/16 per warp
+    static constexpr int NU = VS / 16;
     static_assert(8 % MT == 0 && NTS % WPM == 0, "state tiles over 8 warps");
+    static_assert(STAGE % 16 == 0 && OFF_ST % 16 == 0, "16-byte copies");
 };
 
 template <int DK, int DV>
@@ -210,8 +221,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int lr = lane >> 2, lc = lane & 3;
-    const int64_t bh = blockIdx.x, b = bh / H, h = bh % H;
-    float *gm = reinterpret_cast<float *>(smem + S::OFF_GM);
+    const int64_t bh = blockIdx.x / S::NSL, b = bh / H, h = bh % H;
+    const int v0 = (int)(blockIdx.x % S::NSL) * VS;  // this CTA's rows of the state
 
     // state tiles of this warp: rows 16 ms + (lr, lr + 8), columns 8 (ns0 + n) + 2 lc (+1)
     const int ms = warp % S::MT, ns0 = (warp / S::MT) * S::NPW;
@@ -222,16 +233,52 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = ms * 16 + lr + (e >> 1) * 8, c = (ns0 + n) * 8 + 2 * lc + (e & 1);
-            st[n][e] = sin ? sin[r * DK + c] : 0.f;
+            st[n][e] = sin ? sin[(v0 + r) * DK + c] : 0.f;
         }
     // U / O tiles of this warp: rows 16 mu + (lr, lr + 8), columns 8 (nu0 + n) + 2 lc (+1)
     const int mu = warp & 3, nu0 = (warp >> 2) * S::NU;
+
+    // a chunk's operands into stage stg: W, P and g K from its workspace record,
+    // Q from the queries, gamma
+    auto prefetch = [&](int chn, int stg) {
+        const uint8_t *rec = ws + (size_t)(bh * n_ch + chn) * W::BYTES;
+        const int64_t t0 = (int64_t)chn * C;
+        uint8_t *sb = smem + S::OFF_ST + stg * S::STAGE;
+        for (int i = tid; i < C * (DK / 8); i += THREADS) {
+            const int t = i / (DK / 8), c8 = i % (DK / 8);
+            const int64_t tok = t0 + t;
+            const size_t ro = (size_t)(t * DK + c8 * 8) * 2;
+            const int so = t * S::WSTR + c8 * 16;
+            cp_async16(smem_u32(sb + S::WH + so), rec + W::OFF_WH + ro, 16);
+            cp_async16(smem_u32(sb + S::WL + so), rec + W::OFF_WL + ro, 16);
+            cp_async16(smem_u32(sb + S::KH + so), rec + W::OFF_KH + ro, 16);
+            cp_async16(smem_u32(sb + S::KL + so), rec + W::OFF_KL + ro, 16);
+            cp_async16(smem_u32(sb + S::Q + so),
+                       q + ((b * T + (tok < T ? tok : 0)) * H + h) * DK + c8 * 8,
+                       tok < T ? 16 : 0);
+        }
+        for (int i = tid; i < C * (C / 8); i += THREADS) {
+            const int t = i / (C / 8), c8 = i % (C / 8);
+            const size_t ro = (size_t)(t * C + c8 * 8) * 2;
+            cp_async16(smem_u32(sb + S::PH + t * S::PSTR + c8 * 16), rec + W::OFF_PH + ro, 16);
+            cp_async16(smem_u32(sb + S::PL + t * S::PSTR + c8 * 16), rec + W::OFF_PL + ro, 16);
+        }
+        for (int i = tid; i < C / 4; i += THREADS)
+            cp_async16(smem_u32(sb + S::GM + i * 16), rec + W::OFF_G + i * 16, 16);
+        cp_async_commit();
+    };
+    if (n_ch > 0) prefetch(0, 0);
 
 #pragma unroll 1
     for (int ch = 0; ch < n_ch; ++ch) {
         const int64_t t0 = (int64_t)ch * C;
         const uint8_t *rec = ws + (size_t)(bh * n_ch + ch) * W::BYTES;
-        // ---- the state as bf16 hi + lo; the chunk's operands -----------------
+        const uint8_t *sb = smem + S::OFF_ST + (ch & 1) * S::STAGE;
+        const float *gm = reinterpret_cast<const float *>(sb + S::GM);
+        // the next chunk's operands go into the other stage, free since the
+        // previous chunk ended
+        if (ch + 1 < n_ch) prefetch(ch + 1, (ch + 1) & 1);
+        // ---- the state as bf16 hi + lo --------------------------------------
 #pragma unroll
         for (int n = 0; n < S::NPW; ++n)
 #pragma unroll
@@ -245,46 +292,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 *reinterpret_cast<uint32_t *>(smem + S::OFF_SL + r * S::SSTR + c * 2) =
                     (uint32_t)l0 | ((uint32_t)l1 << 16);
             }
-        for (int i = tid; i < C * (DK / 8); i += THREADS) {
-            const int t = i / (DK / 8), c8 = i % (DK / 8);
-            const int64_t tok = t0 + t;
-            cp_async16(smem_u32(smem + S::OFF_WH + t * S::WSTR + c8 * 16),
-                       rec + W::OFF_WH + (t * DK + c8 * 8) * 2, 16);
-            cp_async16(smem_u32(smem + S::OFF_WL + t * S::WSTR + c8 * 16),
-                       rec + W::OFF_WL + (t * DK + c8 * 8) * 2, 16);
-            cp_async16(smem_u32(smem + S::OFF_Q + t * S::WSTR + c8 * 16),
-                       q + ((b * T + (tok < T ? tok : 0)) * H + h) * DK + c8 * 8,
-                       tok < T ? 16 : 0);
-        }
-        for (int i = tid; i < C * (C / 8); i += THREADS) {
-            const int t = i / (C / 8), c8 = i % (C / 8);
-            cp_async16(smem_u32(smem + S::OFF_PH + t * S::PSTR + c8 * 16),
-                       rec + W::OFF_PH + (t * C + c8 * 8) * 2, 16);
-            cp_async16(smem_u32(smem + S::OFF_PL + t * S::PSTR + c8 * 16),
-                       rec + W::OFF_PL + (t * C + c8 * 8) * 2, 16);
-        }
-        cp_async_commit();
-        const float *gg = reinterpret_cast<const float *>(rec + W::OFF_G);
-        if (tid < C) gm[tid] = gg[tid];
-        for (int i = tid; i < C * (DK / 2); i += THREADS) {  // g_t k_t as hi + lo
-            const int t = i / (DK / 2), c2 = i % (DK / 2);
-            const int64_t tok = t0 + t;
-            float k0 = 0.f, k1 = 0.f;
-            if (tok < T) {
-                const uint32_t kv = *reinterpret_cast<const uint32_t *>(
-                    k + ((b * T + tok) * H + h) * DK + 2 * c2);
-                k0 = bf16_lo(kv) * gg[C + t];
-                k1 = bf16_hi(kv) * gg[C + t];
-            }
-            uint16_t h0, l0, h1, l1;
-            split_bf16(k0, h0, l0);
-            split_bf16(k1, h1, l1);
-            *reinterpret_cast<uint32_t *>(smem + S::OFF_KH + t * S::WSTR + c2 * 4) =
-                (uint32_t)h0 | ((uint32_t)h1 << 16);
-            *reinterpret_cast<uint32_t *>(smem + S::OFF_KL + t * S::WSTR + c2 * 4) =
-                (uint32_t)l0 | ((uint32_t)l1 << 16);
-        }
-        cp_async_wait<0>();
+        if (ch + 1 < n_ch)
+            cp_async_wait<1>();  // this chunk's group; the next one may stay in flight
+        else
+            cp_async_wait<0>();
         __syncthreads();
 
         // ---- U = Ut - W S0^T and O1 = Q S0^T (rows t, columns v; K = DK) ------
@@ -301,9 +312,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t wh[4], wl[4], qa[4];
             const int ar = mu * 16 + (lane & 15);
             const int acol = (ks * 16) * 2 + (lane >> 4) * 16;
-            ldmatrix_x4(smem_u32(smem + S::OFF_WH + ar * S::WSTR + acol), wh[0], wh[1], wh[2], wh[3]);
-            ldmatrix_x4(smem_u32(smem + S::OFF_WL + ar * S::WSTR + acol), wl[0], wl[1], wl[2], wl[3]);
-            ldmatrix_x4(smem_u32(smem + S::OFF_Q + ar * S::WSTR + acol), qa[0], qa[1], qa[2], qa[3]);
+            ldmatrix_x4(smem_u32(sb + S::WH + ar * S::WSTR + acol), wh[0], wh[1], wh[2], wh[3]);
+            ldmatrix_x4(smem_u32(sb + S::WL + ar * S::WSTR + acol), wl[0], wl[1], wl[2], wl[3]);
+            ldmatrix_x4(smem_u32(sb + S::Q + ar * S::WSTR + acol), qa[0], qa[1], qa[2], qa[3]);
 #pragma unroll
             for (int n = 0; n < S::NU; ++n) {
                 // B = S0^T (k x v) from the state rows v (k contiguous): no transpose
@@ -325,7 +336,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int t = mu * 16 + lr + (e >> 1) * 8, c = (nu0 + n) * 8 + 2 * lc + (e & 1);
-                u[n][e] = ut[t * DV + c] - u[n][e];
+                u[n][e] = ut[t * DV + v0 + c] - u[n][e];
                 ov[n][e] *= gm[t];
             }
         // U to shared memory as hi + lo, rows t
@@ -350,8 +361,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t ph[4], pl[4];
             const int ar = mu * 16 + (lane & 15);
             const int acol = (ks * 16) * 2 + (lane >> 4) * 16;
-            ldmatrix_x4(smem_u32(smem + S::OFF_PH + ar * S::PSTR + acol), ph[0], ph[1], ph[2], ph[3]);
-            ldmatrix_x4(smem_u32(smem + S::OFF_PL + ar * S::PSTR + acol), pl[0], pl[1], pl[2], pl[3]);
+            ldmatrix_x4(smem_u32(sb + S::PH + ar * S::PSTR + acol), ph[0], ph[1], ph[2], ph[3]);
+            ldmatrix_x4(smem_u32(sb + S::PL + ar * S::PSTR + acol), pl[0], pl[1], pl[2], pl[3]);
 #pragma unroll
             for (int n = 0; n < S::NU; ++n) {
                 // B = U (tokens x v), rows t (v contiguous): transposed load
@@ -371,7 +382,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int e = 0; e < 4; ++e) {
                 const int t = mu * 16 + lr + (e >> 1) * 8, c = (nu0 + n) * 8 + 2 * lc + (e & 1);
                 const int64_t tok = t0 + t;
-                if (tok < T) o[((b * T + tok) * H + h) * DV + c] = ov[n][e];
+                if (tok < T) o[((b * T + tok) * H + h) * DV + v0 + c] = ov[n][e];
             }
 
         // ---- S = gamma_{C-1} S0 + U^T (g K) (rows v, columns k; K = tokens) ---
@@ -394,8 +405,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int br = ks * 16 + (lane & 15);
                 const int bcol = (ns0 + n) * 16;
                 uint32_t kh0, kh1, kl0, kl1;
-                ldmatrix_x2_trans(smem_u32(smem + S::OFF_KH + br * S::WSTR + bcol), kh0, kh1);
-                ldmatrix_x2_trans(smem_u32(smem + S::OFF_KL + br * S::WSTR + bcol), kl0, kl1);
+                ldmatrix_x2_trans(smem_u32(sb + S::KH + br * S::WSTR + bcol), kh0, kh1);
+                ldmatrix_x2_trans(smem_u32(sb + S::KL + br * S::WSTR + bcol), kl0, kl1);
                 mma_bf16_16816(st[n], ah[0], ah[1], ah[2], ah[3], kh0, kh1);
                 mma_bf16_16816(st[n], ah[0], ah[1], ah[2], ah[3], kl0, kl1);
                 mma_bf16_16816(st[n], al[0], al[1], al[2], al[3], kh0, kh1);
@@ -409,7 +420,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = ms * 16 + lr + (e >> 1) * 8, c = (ns0 + n) * 8 + 2 * lc + (e & 1);
-            sout[r * DK + c] = st[n][e];
+            sout[(v0 + r) * DK + c] = st[n][e];
         }
 }
 
@@ -432,8 +443,8 @@ static cudaError_t launch(const uint16_t *q, const uint16_t *k, const uint16_t *
     auto k2 = gdn_chunk_scan<DK, DV>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(k2), ScanCfg<DK, DV>::BYTES);
     if (e != cudaSuccess) return e;
-    k2<<<(unsigned)bhs, THREADS, ScanCfg<DK, DV>::BYTES, s>>>(q, k, state_in, T, H, n_ch, ws, o,
-                                                               state_out);
+    k2<<<(unsigned)(bhs * ScanCfg<DK, DV>::NSL), THREADS, ScanCfg<DK, DV>::BYTES, s>>>(
+        q, k, state_in, T, H, n_ch, ws, o, state_out);
     return cudaGetLastError();
 }
 

@@ -383,7 +383,7 @@ QSA_API qsa_status_t qsa_gdn_prefill(const qsa_bf16_t *q, const qsa_bf16_t *k,
  * operands split into bf16 high and low parts (about 2^-16 relative per
  * product).  Same arguments and layouts as qsa_gdn_prefill, plus a caller
  * workspace of qsa_gdn_prefill_chunked_workspace_size bytes (256-byte aligned;
- * per (sequence, head, chunk) the chunk's solve: 80.5 KiB at dk = dv = 128).
+ * per (sequence, head, chunk) the chunk's solve: 112.5 KiB at dk = dv = 128).
  * Returns QSA_ERR_WORKSPACE if it is missing, too small or misaligned.
  */
 QSA_API size_t qsa_gdn_prefill_chunked_workspace_size(int B, int64_t T, int H, int dk, int dv);

@@ -178,8 +178,8 @@ def test_gdn_validation(lib):
     assert dec(st=_nullp()) == INVALID
     assert dec(dv=32) == UNSUPPORTED
     # the chunked prefill: its workspace size, then the same checks plus the workspace
-    assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 64, 4, 128, 128) == 256 + 4 * 82432
-    assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 65, 4, 64, 64) == 256 + 2 * 4 * 49664
+    assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 64, 4, 128, 128) == 256 + 4 * 115200
+    assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 65, 4, 64, 64) == 256 + 2 * 4 * 66048
     assert lib.qsa_gdn_prefill_chunked_workspace_size(1, 64, 4, 96, 128) == SIZE_MAX
     big = 1 << 24
     chk = lambda **kw: lib.qsa_gdn_prefill_chunked(*dict(dict(
