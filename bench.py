@@ -819,7 +819,7 @@ def main():
     }
     barrier(world)
     if not args.no_e2e:
-        e2e_ms, h2d, d2h = e2e_prefill(qsa, w, x, device, min(args.steps, 5))
+        e2e_ms, h2d, d2h = e2e_prefill(qsa, w, x, device, args.steps)
         e2e_ms = max_over_ranks(e2e_ms, world, device)
         line["e2e"] = {"value": world * w.B * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
