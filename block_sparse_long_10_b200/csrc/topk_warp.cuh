@@ -224,11 +224,6 @@ QSA_DEVICE uint32_t warp_kth_largest_narrow(const KeyT *buf, int n, int K, uint3
     }
 }
 
-QSA_DEVICE uint32_t warp_kth_largest_u32(const uint32_t *buf, int n, int K, uint32_t *hist,
-                                         int lane) {
-    return warp_kth_largest_narrow<uint32_t>(buf, n, K, hist, lane);
-}
-
 // The K-th largest of n <= 32 R unique 64-bit keys in shared memory
 // (1 <= K <= n) with the high words held in registers: the K-th largest high
 // word t is built bit by bit from the top (keep a bit when at least K high
