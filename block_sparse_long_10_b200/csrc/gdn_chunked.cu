@@ -14,9 +14,11 @@
 // Two kernels:
 //   gdn_chunk_prep  one CTA per (sequence, head, chunk), all in parallel: the
 //                   gates' log prefix sums, A and P from the chunk's dot
-//                   products, the triangular solve for [Ut | W] by forward
-//                   substitution (fp32 on CUDA cores), written to the
-//                   workspace (W and P as bf16 high + low parts);
+//                   products K K^T and Q K^T (mma.sync: bf16 products, fp32
+//                   sums), the triangular solve for [Ut | W] by forward
+//                   substitution in fp32 (one column per thread, held in
+//                   registers: columns do not depend on one another), written
+//                   to the workspace (W and P as bf16 high + low parts);
 //   gdn_chunk_scan  per (sequence, head), VS = 16 rows of the state per CTA
 //                   (the rows are independent: U, O and the state update of a
 //                   row slice need only that slice), each CTA walking its chunks
@@ -56,40 +58,55 @@ QSA_DEVICE void split_bf16(float x, uint16_t &hi, uint16_t &lo) {
 template <int DK, int DV>
 struct PrepCfg {
     static constexpr int NX = DV + DK;                  // columns of [Ut | W]
-    static constexpr int OFF_K = 0;                     // [C][DK + 1] fp32
-    static constexpr int OFF_Q = OFF_K + C * (DK + 1);  // [C][DK + 1] fp32
-    static constexpr int OFF_X = OFF_Q + C * (DK + 1);  // [C][NX] fp32
-    static constexpr int OFF_A = OFF_X + C * NX;        // [C][C + 1] fp32
-    static constexpr int OFF_L = OFF_A + C * (C + 1);   // log prefix [C], beta [C]
-    static constexpr int FLOATS = OFF_L + 2 * C;
-    static constexpr int BYTES = FLOATS * 4;
+    static constexpr int KSTR = DK * 2 + 16;            // K, Q rows (bf16), padded: bytes
+    static constexpr int ASTR = C + 4;                  // A rows (fp32), 16-byte aligned
+    static constexpr int OFF_K = 0;                     // [C][KSTR] bytes
+    static constexpr int OFF_Q = OFF_K + C * KSTR;      // [C][KSTR] bytes
+    static constexpr int OFF_A = OFF_Q + C * KSTR;      // [C][ASTR] fp32
+    static constexpr int OFF_L = OFF_A + C * ASTR * 4;  // log prefix, beta, gamma, g: [C] each
+    static constexpr int BYTES = OFF_L + 4 * C * 4;
+    static_assert(NX <= THREADS, "one column of [Ut | W] per thread");
+    static_assert(KSTR % 16 == 0 && OFF_A % 16 == 0, "16-byte rows");
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 2)
     gdn_chunk_prep(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    const uint16_t *__restrict__ v, const float *__restrict__ alpha,
                    const float *__restrict__ beta, int64_t T, int H, int n_ch,
                    uint8_t *__restrict__ ws) {
     using P = PrepCfg<DK, DV>;
     using W = Ws<DK, DV>;
-    extern __shared__ __align__(16) float sm[];
-    float *Ks = sm + P::OFF_K, *Qs = sm + P::OFF_Q, *X = sm + P::OFF_X, *Am = sm + P::OFF_A;
-    float *ell = sm + P::OFF_L, *bet = ell + C;
-    const int tid = threadIdx.x, lane = tid & 31;
+    extern __shared__ __align__(128) uint8_t smp[];
+    float *As = reinterpret_cast<float *>(smp + P::OFF_A);
+    float *ell = reinterpret_cast<float *>(smp + P::OFF_L), *bet = ell + C;
+    float *gam = bet + C, *gl = gam + C;  // gamma_t, gamma_{C-1} / gamma_t
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lr = lane >> 2, lc = lane & 3;
     const int ch = blockIdx.x % n_ch;
     const int64_t bh = blockIdx.x / n_ch;  // b * H + h
     const int64_t b = bh / H, h = bh % H;
     const int64_t t0 = (int64_t)ch * C;
     uint8_t *rec = ws + (size_t)blockIdx.x * W::BYTES;
+    auto kval = [&](int t, int d) {  // the chunk's key t, dimension d
+        return __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(
+                                   smp + P::OFF_K + t * P::KSTR + d * 2)
+                               << 16);
+    };
 
-    // the chunk's keys, queries, values (v scaled by beta into X's first DV columns)
-    for (int i = tid; i < C * DK; i += THREADS) {
-        const int t = i / DK, d = i % DK;
+    // the chunk's keys and queries as bf16 rows (zeros past the sequence)
+    constexpr int CPR = DK / 8;  // 16-byte pieces per row
+    for (int i = tid; i < C * CPR; i += THREADS) {
+        const int t = i / CPR, c = i % CPR;
         const int64_t tok = t0 + t;
-        const int64_t off = ((b * T + tok) * H + h) * DK + d;
-        Ks[t * (DK + 1) + d] = tok < T ? __uint_as_float((uint32_t)k[off] << 16) : 0.f;
-        Qs[t * (DK + 1) + d] = tok < T ? __uint_as_float((uint32_t)q[off] << 16) : 0.f;
+        uint4 kv = make_uint4(0u, 0u, 0u, 0u), qv = kv;
+        if (tok < T) {
+            const int64_t off = ((b * T + tok) * H + h) * DK + c * 8;
+            kv = *reinterpret_cast<const uint4 *>(k + off);
+            qv = *reinterpret_cast<const uint4 *>(q + off);
+        }
+        *reinterpret_cast<uint4 *>(smp + P::OFF_K + t * P::KSTR + c * 16) = kv;
+        *reinterpret_cast<uint4 *>(smp + P::OFF_Q + t * P::KSTR + c * 16) = qv;
     }
     if (tid < 32) {  // gates: the log prefix of alpha (two tokens per lane), beta
         float la[2];
@@ -110,72 +127,138 @@ __global__ void __launch_bounds__(THREADS)
         const float excl = run - (la[0] + la[1]);
         ell[lane * 2] = excl + la[0];
         ell[lane * 2 + 1] = excl + la[0] + la[1];
+        __syncwarp();
+        const float last = ell[C - 1];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int t = lane * 2 + e;
+            gam[t] = expf(ell[t]);
+            gl[t] = expf(last - ell[t]);
+        }
     }
     __syncthreads();
-    for (int i = tid; i < C * DV; i += THREADS) {
-        const int t = i / DV, d = i % DV;
-        const int64_t tok = t0 + t;
-        const float vv =
-            tok < T ? __uint_as_float((uint32_t)v[((b * T + tok) * H + h) * DV + d] << 16) : 0.f;
-        X[t * P::NX + d] = bet[t] * vv;
-    }
-    for (int i = tid; i < C * DK; i += THREADS) {
-        const int t = i / DK, d = i % DK;
-        X[t * P::NX + DV + d] = bet[t] * expf(ell[t]) * Ks[t * (DK + 1) + d];
-    }
-    // A (strictly lower) and P (lower, with the diagonal): dot products
-    for (int i = tid; i < C * C; i += THREADS) {
-        const int t = i / C, j = i % C;
-        float a = 0.f, p = 0.f;
-        if (j <= t) {
-            float dk_ = 0.f, dq_ = 0.f;
-#pragma unroll 8
-            for (int d = 0; d < DK; ++d) {
-                const float kj = Ks[j * (DK + 1) + d];
-                dk_ = fmaf(Ks[t * (DK + 1) + d], kj, dk_);
-                dq_ = fmaf(Qs[t * (DK + 1) + d], kj, dq_);
+
+    // A (strictly lower) and P (lower, with the diagonal) from the chunk's dot
+    // products K K^T and Q K^T on mma.sync (bf16 products, fp32 sums).  Warp
+    // pair mt = warp / 2 takes rows 16 mt .. 16 mt + 15 and the 2 (mt + 1)
+    // eight-column tiles of the lower triangle there, mt + 1 per warp.
+    {
+        const int mt = warp >> 1, half = warp & 1, ntn = mt + 1;
+        float accA[4][4], accP[4][4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) accA[n][e] = accP[n][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+            const int ar = mt * 16 + (lane & 15), acol = ks * 32 + (lane >> 4) * 16;
+            uint32_t ak[4], aq[4];
+            ldmatrix_x4(smem_u32(smp + P::OFF_K + ar * P::KSTR + acol), ak[0], ak[1], ak[2], ak[3]);
+            ldmatrix_x4(smem_u32(smp + P::OFF_Q + ar * P::KSTR + acol), aq[0], aq[1], aq[2], aq[3]);
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                if (n < ntn) {
+                    const int nt = half * ntn + n;
+                    const int br = nt * 8 + (lane & 7), bcol = ks * 32 + ((lane >> 3) & 1) * 16;
+                    uint32_t b0, b1;
+                    ldmatrix_x2(smem_u32(smp + P::OFF_K + br * P::KSTR + bcol), b0, b1);
+                    mma_bf16_16816(accA[n], ak[0], ak[1], ak[2], ak[3], b0, b1);
+                    mma_bf16_16816(accP[n], aq[0], aq[1], aq[2], aq[3], b0, b1);
+                }
             }
-            const float gr = expf(ell[t] - ell[j]);
-            if (j < t) a = bet[t] * gr * dk_;
-            p = gr * dq_;
         }
-        Am[t * (C + 1) + j] = a;
-        // P goes straight to the workspace as hi + lo
-        uint16_t ph, pl;
-        split_bf16(p, ph, pl);
-        reinterpret_cast<uint16_t *>(rec + W::OFF_PH)[t * C + j] = ph;
-        reinterpret_cast<uint16_t *>(rec + W::OFF_PL)[t * C + j] = pl;
+        uint32_t *ph2 = reinterpret_cast<uint32_t *>(rec + W::OFF_PH);
+        uint32_t *pl2 = reinterpret_cast<uint32_t *>(rec + W::OFF_PL);
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            if (n < ntn) {
+                const int nt = half * ntn + n;
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {  // rows lr, lr + 8 of the tile
+                    const int t = mt * 16 + lr + hr * 8;
+                    uint16_t phv[2], plv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int j = nt * 8 + 2 * lc + e;
+                        float a = 0.f, pv = 0.f;
+                        if (j <= t) {
+                            const float gr = expf(ell[t] - ell[j]);
+                            if (j < t) a = bet[t] * gr * accA[n][hr * 2 + e];
+                            pv = gr * accP[n][hr * 2 + e];
+                        }
+                        As[t * P::ASTR + j] = a;
+                        split_bf16(pv, phv[e], plv[e]);
+                    }
+                    // P goes straight to the workspace as hi + lo
+                    ph2[(t * C + nt * 8 + 2 * lc) >> 1] = (uint32_t)phv[0] | ((uint32_t)phv[1] << 16);
+                    pl2[(t * C + nt * 8 + 2 * lc) >> 1] = (uint32_t)plv[0] | ((uint32_t)plv[1] << 16);
+                }
+            }
+        }
+        // P above the diagonal blocks (no tile computed there) is zero
+        for (int i = tid; i < C * C / 2; i += THREADS) {
+            const int t = i / (C / 2), j = (i % (C / 2)) * 2;
+            if (j >= (t / 16) * 16 + 16) {
+                ph2[i] = 0u;
+                pl2[i] = 0u;
+            }
+        }
     }
     __syncthreads();
-    // forward substitution: row t of [Ut | W] minus the earlier rows it depends on
-    for (int t = 1; t < C; ++t) {
-        for (int col = tid; col < P::NX; col += THREADS) {
-            float acc = X[t * P::NX + col];
-            for (int j = 0; j < t; ++j) acc = fmaf(-Am[t * (C + 1) + j], X[j * P::NX + col], acc);
-            X[t * P::NX + col] = acc;
+
+    // forward substitution, one column of [Ut | W] per thread, held in
+    // registers (a column depends only on itself and A): row t minus the
+    // earlier rows it depends on, in the order j = 0 .. t - 1
+    if (tid < P::NX) {
+        const int col = tid;
+        float x[C];
+        if (col < DV) {  // beta v
+#pragma unroll
+            for (int t = 0; t < C; ++t) {
+                const int64_t tok = t0 + t;
+                const float vv =
+                    tok < T ? __uint_as_float((uint32_t)v[((b * T + tok) * H + h) * DV + col] << 16)
+                            : 0.f;
+                x[t] = bet[t] * vv;
+            }
+        } else {  // beta gamma k
+#pragma unroll
+            for (int t = 0; t < C; ++t) x[t] = bet[t] * gam[t] * kval(t, col - DV);
         }
-        __syncthreads();
-    }
-    for (int i = tid; i < C * DV; i += THREADS) {
-        const int t = i / DV, d = i % DV;
-        reinterpret_cast<float *>(rec + W::OFF_U)[t * DV + d] = X[t * P::NX + d];
-    }
-    for (int i = tid; i < C * DK; i += THREADS) {
-        const int t = i / DK, d = i % DK;
-        uint16_t wh, wl;
-        split_bf16(X[t * P::NX + DV + d], wh, wl);
-        reinterpret_cast<uint16_t *>(rec + W::OFF_WH)[t * DK + d] = wh;
-        reinterpret_cast<uint16_t *>(rec + W::OFF_WL)[t * DK + d] = wl;
+#pragma unroll
+        for (int t = 1; t < C; ++t) {
+            float acc = x[t];
+            const float4 *arow = reinterpret_cast<const float4 *>(As + t * P::ASTR);
+#pragma unroll
+            for (int j4 = 0; j4 < (t + 3) / 4; ++j4) {
+                const float4 a4 = arow[j4];
+                acc = fmaf(-a4.x, x[4 * j4], acc);
+                if (4 * j4 + 1 < t) acc = fmaf(-a4.y, x[4 * j4 + 1], acc);
+                if (4 * j4 + 2 < t) acc = fmaf(-a4.z, x[4 * j4 + 2], acc);
+                if (4 * j4 + 3 < t) acc = fmaf(-a4.w, x[4 * j4 + 3], acc);
+            }
+            x[t] = acc;
+        }
+        if (col < DV) {
+            float *u = reinterpret_cast<float *>(rec + W::OFF_U);
+#pragma unroll
+            for (int t = 0; t < C; ++t) u[t * DV + col] = x[t];
+        } else {
+            uint16_t *wh = reinterpret_cast<uint16_t *>(rec + W::OFF_WH);
+            uint16_t *wl = reinterpret_cast<uint16_t *>(rec + W::OFF_WL);
+#pragma unroll
+            for (int t = 0; t < C; ++t) split_bf16(x[t], wh[t * DK + col - DV], wl[t * DK + col - DV]);
+        }
     }
     if (tid < C) {
         float *g = reinterpret_cast<float *>(rec + W::OFF_G);
-        g[tid] = expf(ell[tid]);                  // gamma_t
-        g[C + tid] = expf(ell[C - 1] - ell[tid]); // gamma_{C-1} / gamma_t
+        g[tid] = gam[tid];
+        g[C + tid] = gl[tid];
     }
     for (int i = tid; i < C * DK; i += THREADS) {  // g_t k_t, the state update's operand
         const int t = i / DK, d = i % DK;
         uint16_t kh, kl;
-        split_bf16(expf(ell[C - 1] - ell[t]) * Ks[t * (DK + 1) + d], kh, kl);
+        split_bf16(gl[t] * kval(t, d), kh, kl);
         reinterpret_cast<uint16_t *>(rec + W::OFF_KH)[t * DK + d] = kh;
         reinterpret_cast<uint16_t *>(rec + W::OFF_KL)[t * DK + d] = kl;
     }
